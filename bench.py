@@ -1,0 +1,436 @@
+"""Benchmark of the batched Muon step + batched EMA on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload 6]
+
+One step = muon_step_batched over the 66 matrices of the 11L x 512d GPT
+(K = 5 fixed-quintic Newton-Schulz steps, momentum 0.99, lr 0.022, wd 0.105,
+MuonEq-R) followed by ema_update_batched over every parameter of the same
+model (38,071,388 fp32, decay 0.9965): every row of the hot path.  Inputs are
+synthetic (seeded), resident in HBM and larger than L2 (0.9 GB of state).
+
+For N > 1 it runs under torch.distributed.run, one rank per GPU; each rank
+steps its own replica (weak scaling, no collective on the data path); the
+time is the max over ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (rank 0
+only) on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from muon_optimizer_step_02_b200 import workloads as wl  # noqa: E402
+
+METRIC = ("Muon steps/s (66-matrix 11L×512d set); NS TFLOP/s & EMA "
+          "GB/s as % of B200 peak")
+UNIT = "steps/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+                  "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------
+# clocks
+# --------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            self.path = f"/tmp/muonb200_clocks_{os.getpid()}.csv"
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu)], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+        os.remove(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# our implementation
+# --------------------------------------------------------------------------
+class Workload:
+    """Device state of one replica of the benchmark workload."""
+
+    def __init__(self, w: wl.Workload, seed: int):
+        import torch
+        from muon_optimizer_step_02_b200 import binding as B
+        self.B = B
+        self.w = w
+        self.plan = B.MuonPlan(w.shapes, max_ns_steps=len(w.coeffs))
+        self.ws = self.plan.alloc_workspace()
+        self.W = [torch.from_numpy(wl.weight(w, i, seed)).cuda()
+                  for i in range(w.n_mats)]
+        self.M = [torch.zeros_like(x) for x in self.W]
+        self.G_host = [torch.from_numpy(wl.grad_bits(w, i, 0, seed)
+                                        .view(np.int16)).view(torch.bfloat16)
+                       for i in range(w.n_mats)]
+        self.G = [g.cuda() for g in self.G_host]
+        self.scales = wl.update_scales(w)
+        # EMA over every parameter: the matrices (their current W) plus the
+        # non-matrix tensors.
+        self.extra = []
+        for j, n in enumerate(w.ema_extra_numels):
+            _, p = wl.ema_pair(w, w.n_mats + j, seed)
+            self.extra.append(torch.from_numpy(p).cuda())
+        self.E = [x.clone() for x in self.W] + [x.clone() for x in self.extra]
+        self.P = [x.view(-1) for x in self.W] + self.extra
+        self.E = [e.view(-1) for e in self.E]
+
+    def step(self):
+        self.plan.step(self.W, self.M, self.G, self.w.hyper, self.w.coeffs,
+                       self.ws, update_scales=self.scales)
+        if self.w.ema_decay is not None:
+            self.B.ema_update_batched(self.E, self.P, self.w.ema_decay)
+
+    def launches_per_step(self) -> int:
+        n = self.B.step_launches(len(self.w.coeffs))
+        if self.w.ema_decay is not None:
+            n += self.B.ema_launches(len(self.E))
+        return n
+
+    def ns_flops_by_kind(self):
+        gram = sum(2 * min(r, c) ** 2 * max(r, c) for r, c in self.w.shapes)
+        poly = sum(2 * min(r, c) ** 3 for r, c in self.w.shapes)
+        return {"gram": gram, "poly": poly, "apply": gram}
+
+    def state_bytes(self):
+        elems = self.w.numel()
+        return {"prologue": 12 * elems,  # G 2 + M 4+4 + X~ 2
+                "ema": 12 * sum(self.w.ema_numels())}
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    w = wl.workload(args.workload)
+    rep = Workload(w, seed=1337 + rank)
+    stream = torch.cuda.current_stream()
+    peaks, peak_src = load_peaks()
+
+    for _ in range(args.warmup):
+        rep.step()
+    torch.cuda.synchronize()
+    assert rep.plan.last_error() == 0
+
+    # ---- timed region: device time with CUDA events, per-launch events on
+    # the launching stream for the roofline.
+    rep.plan.set_timing(True)
+    rep.plan.timing_read()  # reset
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        rep.step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    phase = rep.plan.timing_read()
+    rep.plan.set_timing(False)
+    if rep.plan.last_error() != 0:
+        raise RuntimeError("device-side error during the timed region")
+    if world > 1:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * args.steps / (ms / 1e3)
+
+    # ---- EMA time (own events, the EMA kernel is launched on this stream)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    ema_ms = None
+    if w.ema_decay is not None:
+        reps = max(3, args.steps // 4)
+        e0.record(stream)
+        for _ in range(reps):
+            rep.B.ema_update_batched(rep.E, rep.P, w.ema_decay)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ema_ms = e0.elapsed_time(e1) / reps
+
+    # ---- end to end through the public API with host buffers: pinned
+    # gradients copied in every step, the status word read back every step.
+    G_pin = [g.pin_memory() for g in rep.G_host]
+    h2d = sum(g.numel() * 2 for g in G_pin)
+    e2e_steps = max(3, min(args.steps, 50))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    tt0 = torch.cuda.Event(enable_timing=True)
+    tt1 = torch.cuda.Event(enable_timing=True)
+    tt0.record(stream)
+    for _ in range(e2e_steps):
+        for dst, src in zip(rep.G, G_pin):
+            dst.copy_(src, non_blocking=True)
+        rep.step()
+        if rep.plan.last_error() != 0:   # syncs, reads 4 bytes
+            raise RuntimeError("device-side error in the e2e loop")
+    tt1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = tt0.elapsed_time(tt1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * e2e_steps / (e2e_ms / 1e3)
+
+    if rank != 0:
+        return None
+
+    # ---- roofline of the dominant kernel
+    flops = rep.ns_flops_by_kind()
+    ns_kinds = ("gram", "poly", "apply")
+    dom = max(phase, key=lambda k: phase[k][1])
+    launches_dom, ms_dom = phase[dom]
+    sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    if dom in ns_kinds:
+        per_launch = flops[dom]
+        achieved = per_launch / (ms_dom / launches_dom / 1e3) / 1e12
+        roof = {"kernel": f"ns_gemm ({dom})", "bound": "tensor",
+                "achieved": round(achieved, 2), "peak": sustained,
+                "unit": "TFLOP/s", "frac": round(achieved / sustained, 4),
+                "traffic": None, "peak_source": f"{peak_src} sustained bf16"}
+    else:
+        per_launch = rep.state_bytes()["prologue"]
+        achieved = per_launch / (ms_dom / launches_dom / 1e3) / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": None, "peak_source": f"{peak_src} HBM copy"}
+    ns_ms = sum(phase[k][1] for k in ns_kinds) / args.steps
+    ns_flops = sum(flops[k] for k in ns_kinds) * len(w.coeffs)
+    ns_tflops = ns_flops / (ns_ms / 1e3) / 1e12 if ns_ms > 0 else None
+    pro_ms = phase["prologue"][1] / max(phase["prologue"][0], 1)
+    breakdown = {k: {"launches": v[0], "ms_per_step": round(v[1] / args.steps, 4)}
+                 for k, v in phase.items() if v[0] > 0}
+    ema_gbs = (rep.state_bytes()["ema"] / (ema_ms / 1e3) / 1e9) if ema_ms else None
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16+f32",
+        "data": "synthetic (seeded N(0,0.02) weights, N(0,1e-3) bf16 grads)",
+        "config": {"workload": w.name, "n_mats": w.n_mats,
+                   "matrix_params": w.numel(),
+                   "ema_params": sum(w.ema_numels()),
+                   "ns_steps": len(w.coeffs), "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (0.9 GB of state per step)",
+                   "mode": "eager launches"},
+        "clocks": clk,
+        "e2e": {"value": round(e2e_value, 3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4},
+        "gpu_launches": rep.launches_per_step() * args.steps,
+        "roofline": roof,
+        "ns": {"tflops": round(ns_tflops, 2) if ns_tflops else None,
+               "frac_of_sustained": round(ns_tflops / sustained, 4)
+               if ns_tflops else None, "ms_per_step": round(ns_ms, 4)},
+        "prologue_gbs": round(rep.state_bytes()["prologue"] / (pro_ms / 1e3) / 1e9, 1)
+        if pro_ms > 0 else None,
+        "ema": {"gbs": round(ema_gbs, 1) if ema_gbs else None,
+                "frac": round(ema_gbs / peaks["hbm_gbs"], 4) if ema_gbs else None,
+                "ms": round(ema_ms, 4) if ema_ms else None},
+        "breakdown": breakdown,
+    }
+    return line
+
+
+# --------------------------------------------------------------------------
+# the fp64 oracle on the host cores
+# --------------------------------------------------------------------------
+def oracle_sample(w: wl.Workload, budget_s: float, seed: int = 1337):
+    """Times the oracle on whole layers (6 matrices each, in model order) plus
+    the EMA over the same fraction of the parameters, until about budget_s
+    seconds of CPU work; returns (seconds per full step, description,
+    threads)."""
+    import oracle.muon_oracle as mo
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([d.get("num_threads", 1) for d in threadpool_info()]
+                      or [os.cpu_count()])
+    except Exception:
+        threads = os.cpu_count()
+    hyp = mo.MuonHyper(momentum=w.hyper.momentum, lr=w.hyper.lr,
+                       weight_decay=w.hyper.weight_decay,
+                       eps_row=w.hyper.eps_row, eps_frob=w.hyper.eps_frob,
+                       nesterov=w.hyper.nesterov, eq_r=w.hyper.eq_r)
+    scales = wl.update_scales(w)
+    per_layer = 6 if w.n_mats % 6 == 0 else 1
+    n_groups = w.n_mats // per_layer
+    done, spent = 0, 0.0
+    while done < n_groups and spent < budget_s:
+        idx = range(done * per_layer, (done + 1) * per_layer)
+        ins = [(wl.weight(w, i, seed).astype(np.float64),
+                np.zeros(w.shapes[i]),
+                wl.bf16_bits_to_f32(wl.grad_bits(w, i, 0, seed))
+                .astype(np.float64)) for i in idx]
+        t = time.perf_counter()
+        for (W, M, G), i in zip(ins, idx):
+            mo.muon_step(W, M, G, hyp, w.coeffs, scales[i])
+        spent += time.perf_counter() - t
+        done += 1
+    frac = done / n_groups
+    ema_s = 0.0
+    if w.ema_decay is not None:
+        total = sum(w.ema_numels())
+        n = max(int(total * frac), 1)
+        E = np.random.default_rng(0).standard_normal(n).astype(np.float32) * 0.02
+        P = np.random.default_rng(1).standard_normal(n).astype(np.float32) * 0.02
+        t = time.perf_counter()
+        mo.ema_update(E, P, w.ema_decay)
+        ema_s = time.perf_counter() - t
+    step_s = (spent + ema_s) / frac
+    desc = (f"{done * per_layer} of {w.n_mats} matrices (whole layers) + EMA "
+            f"over the same fraction of {sum(w.ema_numels())} params, "
+            f"extrapolated x{1 / frac:.2f}")
+    return step_s, desc, threads
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return None
+    w = wl.workload(args.workload)
+    budget = float(os.environ.get("MUONB200_ORACLE_BUDGET_S", "20"))
+    times, desc, threads = [], "", os.cpu_count()
+    for _ in range(args.warmup):
+        oracle_sample(w, budget / 4)
+    for _ in range(args.steps):
+        s, desc, threads = oracle_sample(w, budget / max(args.steps, 1))
+        times.append(s)
+    step_s = statistics.mean(times)
+    value = 1.0 / step_s
+    return {
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "impl": "reference", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "n_mats": w.n_mats,
+                   "ns_steps": len(w.coeffs)},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT,
+                         "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 6), "unit": UNIT,
+                "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", type=int, default=6)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if line is None:
+        return
+    if not args.no_cpu_baseline:
+        budget = float(os.environ.get("MUONB200_ORACLE_BUDGET_S", "15"))
+        s, desc, threads = oracle_sample(wl.workload(args.workload), budget)
+        line["cpu_baseline"] = {"value": round(1.0 / s, 6), "unit": UNIT,
+                                "cores": threads, "kind": "oracle",
+                                "sample": desc}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,179 @@
+/*
+ * muon_b200.h -- C ABI of the fused, batched Muon optimizer step and the
+ * batched EMA pass for one NVIDIA B200 (sm_100a).
+ *
+ * What the calls compute (sources are parameter-golf competition pages):
+ *  - muon_step_batched: for every matrix weight W (rows x cols, out x in) with
+ *    bf16 gradient G and fp32 momentum M, one Muon step:
+ *        M' = mu M + G ;  U = G + mu M'   (U = M' without Nesterov)
+ *        U_i <- U_i / (||U_i|| + eps_row)            (MuonEq-R, stored rows)
+ *        X = U^T if rows > cols else U ;  X <- X / (||X||_F + eps_frob)
+ *        K times: A = X X^T ; B = b_k A + c_k A A ; X <- a_k X + B X
+ *        O = X^T if transposed else X
+ *        W' = W (1 - lr wd) - lr scale O
+ *    PR #1584 "Record: Improved Parallel Residuals + Systems Optimization",
+ *    section "Summary" (fused Muon kernel, batched EMA); PR #1396 "Record:
+ *    Combined 3-Layer Recurrence + Parallel Residuals + Polar Express +
+ *    Brotli", table "Techniques Combined" (Polar Express Newton-Schulz with
+ *    4 minimax-optimal steps, MuonEq-R row-norm before NS, WD=0.105);
+ *    PR #1893 "Record: L_ParallelResiduals_UNetSkips_DepthRecur_Muon_
+ *    1.0901", table "Architecture and training stack", row "Optimizer".
+ *    The pages name the steps but print no formulas; the formulas above are
+ *    the readings this library implements.
+ *  - ema_update_batched: E' = d E + (1 - d) P for every parameter tensor
+ *    (PR #1893, same table, row "EMA": EMA_DECAY=0.9965).
+ *
+ * Conventions for every call:
+ *  - Pointers named device point to device memory; pointers to structs and
+ *    arrays of pointers (mats, ema, params, numel, ns_coeffs, hyper) are
+ *    HOST memory read during the call only.
+ *  - The caller owns every buffer.  No call allocates device memory except
+ *    muon_plan_create (a small table owned by the plan until
+ *    muon_plan_destroy).
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and the calls return without synchronising, except
+ *    muon_get_last_error, which synchronises `stream`.
+ *  - Argument, shape and alignment errors are detected on the host and
+ *    returned before anything is enqueued.  Launch failures return
+ *    MUON_ERR_CUDA.  A device-side wait that exceeds its time limit (about one
+ *    second) makes the kernel record an error word, drain its own copies and
+ *    return; muon_get_last_error reports it as MUON_ERR_TIMEOUT.
+ */
+#ifndef MUON_B200_H
+#define MUON_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MUON_OK = 0,
+  MUON_ERR_INVALID_ARG = -1, /* null pointer, bad size, non-finite scalar   */
+  MUON_ERR_UNSUPPORTED = -2, /* shape or step count beyond the plan         */
+  MUON_ERR_ALIGNMENT = -3,   /* a device pointer is not 16-byte aligned      */
+  MUON_ERR_CUDA = -4,        /* CUDA runtime/driver error (launch, encode)   */
+  MUON_ERR_TIMEOUT = -5,     /* a device-side bounded wait ran out           */
+  MUON_ERR_WORKSPACE = -6    /* workspace null, too small or misaligned      */
+} muon_status_t;
+
+/* Opaque plan: matrix shapes, schedule tables and a small device table. */
+typedef struct muon_plan muon_plan_t;
+
+/* A cudaStream_t, passed as an untyped handle. */
+typedef void *muon_stream_t;
+
+/* One matrix of the batch.
+ *  w          device, fp32, rows x cols row-major; read and updated in place.
+ *  momentum   device, fp32, rows x cols row-major; read and updated in place.
+ *  grad_bf16  device, bf16 bit patterns, rows x cols row-major; read only.
+ *  update_out device, fp32, rows x cols row-major, or NULL.  When set it
+ *             receives the orthogonalised update O (before lr and scale).
+ *  rows, cols must equal the shape given to muon_plan_create.
+ *  update_scale  multiplies lr for this matrix (e.g. sqrt(max(1, rows/cols))).
+ *  All non-NULL pointers must be 16-byte aligned. */
+typedef struct {
+  float *w;
+  float *momentum;
+  const uint16_t *grad_bf16;
+  float *update_out;
+  int32_t rows;
+  int32_t cols;
+  float update_scale;
+} muon_matrix_t;
+
+/* Per-call scalars.  momentum in [0, 1); lr, weight_decay finite; eps_row,
+ * eps_frob >= 0 (added to the norms); nesterov, eq_r are 0 or 1. */
+typedef struct {
+  float momentum;
+  float lr;
+  float weight_decay;
+  float eps_row;
+  float eps_frob;
+  int32_t nesterov;
+  int32_t eq_r;
+} muon_hyper_t;
+
+/* Builds a plan for n_mats matrices with the given (host) shapes, for up to
+ * max_ns_steps Newton-Schulz steps per call.  Allocates the plan's device
+ * table on the current device.  rows, cols >= 1; 1 <= n_mats <= 4096;
+ * 0 <= max_ns_steps <= 16.  On success *out owns the plan. */
+muon_status_t muon_plan_create(const int32_t *rows, const int32_t *cols,
+                               int32_t n_mats, int32_t max_ns_steps,
+                               muon_plan_t **out);
+
+/* Bytes of device workspace muon_step_batched needs for this plan: two bf16
+ * copies of every working matrix X (m x n), the bf16 A and B (m x m) of every
+ * matrix, and per-row-block norm partials.  Returns 0 for a NULL plan. */
+size_t muon_plan_workspace_bytes(const muon_plan_t *plan);
+
+/* One Muon step over every matrix of the plan (the definition at the top of
+ * this file).  mats: host array of n_mats entries in plan order.  ns_coeffs:
+ * host array of ns_steps rows (a, b, c); ns_steps in [0, max_ns_steps]; with
+ * 0 steps O is the normalised X.  workspace: device, >= workspace_bytes,
+ * 256-byte aligned; its contents need not be initialised and are clobbered.
+ * Calls on one plan must be ordered (one stream, or synchronised), because
+ * the plan's device table and the workspace are shared.  A call is
+ * deterministic: same inputs give bitwise-equal outputs. */
+muon_status_t muon_step_batched(muon_plan_t *plan, const muon_matrix_t *mats,
+                                const muon_hyper_t *hyper,
+                                const float *ns_coeffs, int32_t ns_steps,
+                                void *workspace, size_t workspace_bytes,
+                                muon_stream_t stream);
+
+/* E' = decay E + (1 - decay) P for n_tensors tensors in one pass.
+ *  ema     host array of device fp32 pointers (updated in place).
+ *  params  host array of device fp32 pointers (read only).
+ *  numel   host array of element counts (>= 0).
+ *  Pointers need 4-byte alignment; 16-byte aligned tensors take the
+ *  vectorised path.  An ema tensor must not overlap another tensor. */
+muon_status_t ema_update_batched(float *const *ema, const float *const *params,
+                                 const int64_t *numel, int32_t n_tensors,
+                                 float decay, muon_stream_t stream);
+
+/* Synchronises `stream`, reads and clears the plan's device error word.
+ * Returns MUON_ERR_TIMEOUT if a kernel gave up on a bounded wait since the
+ * last call, MUON_ERR_CUDA on a CUDA error, MUON_OK otherwise. */
+muon_status_t muon_get_last_error(muon_plan_t *plan, muon_stream_t stream);
+
+/* Static description of a status code. */
+const char *muon_status_string(muon_status_t status);
+
+/* Frees the plan and its device table (synchronises the device first). */
+void muon_plan_destroy(muon_plan_t *plan);
+
+/* Per-kernel timing.  While enabled, muon_step_batched records CUDA events on
+ * `stream` around each launch.  muon_plan_timing_read synchronises and
+ * returns, per launch kind (see muon_kind_t), the number of launches and the
+ * summed milliseconds since the last read, then resets the sums. */
+typedef enum {
+  MUON_KIND_PROLOGUE = 0, /* momentum + MuonEq-R + Frobenius partials      */
+  MUON_KIND_GRAM = 1,     /* A = X X^T                                     */
+  MUON_KIND_POLY = 2,     /* B = b A + c A A                               */
+  MUON_KIND_APPLY = 3,    /* X <- a X + B X (and, last step, W update)     */
+  MUON_KIND_FINAL = 4,    /* ns_steps == 0: W update from the normalised X */
+  MUON_KIND_COUNT = 5
+} muon_kind_t;
+muon_status_t muon_plan_set_timing(muon_plan_t *plan, int32_t enable);
+muon_status_t muon_plan_timing_read(muon_plan_t *plan, int32_t *launches,
+                                    double *ms, int32_t n_kinds);
+
+/* Launch counts of one call with ns_steps steps (for launch accounting). */
+int32_t muon_step_launches(int32_t ns_steps);
+int32_t ema_update_launches(int32_t n_tensors);
+
+/* Test hook: fault 1 makes the tensor-core kernel's load warp skip one
+ * stage of its first tile in block 0, so that the consumer's bounded wait
+ * runs out and the timeout path is exercised.  0 turns it off. */
+muon_status_t muon_plan_set_fault(muon_plan_t *plan, int32_t fault);
+
+/* ABI version (major * 100 + minor). */
+int32_t muon_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUON_B200_H */

@@ -1,0 +1,268 @@
+// K-PRO: the elementwise front of the Muon step, one HBM pass per matrix.
+//
+// Per stored row of every matrix:  M' = mu M + G;  U = G + mu M' (Nesterov);
+// r = ||U||;  X~ = U / (r + eps_row) (MuonEq-R);  X~ is written in bf16 in the
+// working orientation (transposed through shared memory when rows > cols);
+// the Frobenius partial sum of X~ over the work item goes to `partials`.
+//
+// Sources: PR #1893 "Record: L_ParallelResiduals_UNetSkips_DepthRecur_Muon_
+// 1.0901", table "Architecture and training stack", row "Optimizer" (Muon,
+// momentum 0.99); PR #1396 "Record: Combined 3-Layer Recurrence + Parallel
+// Residuals + Polar Express + Brotli", table "Techniques Combined", row
+// "MuonEq-R" (row-norm before NS).
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "muon_types.cuh"
+
+namespace muonb200 {
+
+__device__ __forceinline__ float warp_allreduce_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// Element e of chunk ch for this lane: contiguous 8-element groups on the
+// vector path, lane-strided elements otherwise.
+__device__ __forceinline__ int chunk_pos(bool vec, int ch, int lane, int e) {
+  return vec ? ch * 256 + lane * 8 + e : ch * 256 + e * 32 + lane;
+}
+
+__device__ __forceinline__ void load_g_m(const uint16_t* __restrict__ g,
+                                         const float* __restrict__ mo,
+                                         bool vec, int ch, int lane, int cols,
+                                         float (&gv)[8], float (&mv)[8]) {
+  if (vec) {
+    const int p0 = ch * 256 + lane * 8;
+    if (p0 < cols) {
+      const uint4 graw = __ldcs(reinterpret_cast<const uint4*>(g + p0));
+      const float4 m0 = __ldcs(reinterpret_cast<const float4*>(mo + p0));
+      const float4 m1 = __ldcs(reinterpret_cast<const float4*>(mo + p0 + 4));
+      const uint32_t gw[4] = {graw.x, graw.y, graw.z, graw.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        gv[2 * i] = __uint_as_float(gw[i] << 16);
+        gv[2 * i + 1] = __uint_as_float(gw[i] & 0xFFFF0000u);
+      }
+      mv[0] = m0.x; mv[1] = m0.y; mv[2] = m0.z; mv[3] = m0.w;
+      mv[4] = m1.x; mv[5] = m1.y; mv[6] = m1.z; mv[7] = m1.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) gv[e] = mv[e] = 0.f;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int p = chunk_pos(false, ch, lane, e);
+      gv[e] = p < cols ? bf16_bits_to_float(g[p]) : 0.f;
+      mv[e] = p < cols ? mo[p] : 0.f;
+    }
+  }
+}
+
+__device__ __forceinline__ void store_m(float* __restrict__ mo, bool vec,
+                                        int ch, int lane, int cols,
+                                        const float (&mv)[8]) {
+  if (vec) {
+    const int p0 = ch * 256 + lane * 8;
+    if (p0 < cols) {
+      __stcs(reinterpret_cast<float4*>(mo + p0),
+             make_float4(mv[0], mv[1], mv[2], mv[3]));
+      __stcs(reinterpret_cast<float4*>(mo + p0 + 4),
+             make_float4(mv[4], mv[5], mv[6], mv[7]));
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int p = chunk_pos(false, ch, lane, e);
+      if (p < cols) mo[p] = mv[e];
+    }
+  }
+}
+
+// Writes 8 normalised values of one stored row: straight into X (row-major)
+// or into the shared staging tile for the transposed write-out.
+__device__ __forceinline__ void emit_x(__nv_bfloat16* __restrict__ xrow,
+                                       __nv_bfloat16* __restrict__ srow,
+                                       bool transposed, bool vec, int ch,
+                                       int lane, int cols,
+                                       const float (&x)[8]) {
+  if (vec) {
+    const int p0 = ch * 256 + lane * 8;
+    if (p0 >= cols) return;
+    __nv_bfloat162 h[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    if (!transposed) {
+      *reinterpret_cast<uint4*>(xrow + p0) = *reinterpret_cast<uint4*>(h);
+    } else {
+      // staging rows are (cols + 2) elements: 4-byte aligned only
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<__nv_bfloat162*>(srow + p0 + 2 * i) = h[i];
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int p = chunk_pos(false, ch, lane, e);
+      if (p < cols) {
+        const __nv_bfloat16 v = __float2bfloat16_rn(x[e]);
+        if (!transposed) xrow[p] = v; else srow[p] = v;
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kProThreads)
+muon_prologue_kernel(const MatDev* __restrict__ mats,
+                     const ProItem* __restrict__ items, HyperDev h,
+                     float* __restrict__ partials) {
+  extern __shared__ __align__(16) unsigned char pro_smem[];
+  __shared__ float warp_sums[kProThreads / 32];
+
+  const ProItem it = items[blockIdx.x];
+  const MatDev& md = mats[it.mat];
+  const int cols = md.cols;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool vec = (cols & 7) == 0;
+  const bool tr = md.transposed != 0;
+  const int sld = cols + 2;  // staging row stride (elements)
+  __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(pro_smem);
+  const int nch = (cols + 255) / 256;
+  const float mu = h.mu;
+
+  float fro = 0.f;
+  for (int r = warp; r < it.nrows; r += kProThreads / 32) {
+    const int row = it.row0 + r;
+    const size_t base = static_cast<size_t>(row) * cols;
+    const uint16_t* g = md.g + base;
+    float* mo = md.mom + base;
+    __nv_bfloat16* xrow = tr ? nullptr : md.x[0] + static_cast<size_t>(row) * md.ldx;
+    __nv_bfloat16* srow = tr ? stage + r * sld : nullptr;
+
+    float cache[kProCachedChunks][8];
+    float ss = 0.f;
+    // Pass 1: momentum update, look-ahead, row sum of squares.
+#pragma unroll
+    for (int ch = 0; ch < kProCachedChunks; ++ch) {
+      if (ch < nch) {
+        float gv[8], mv[8];
+        load_g_m(g, mo, vec, ch, lane, cols, gv, mv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float mn = fmaf(mu, mv[e], gv[e]);
+          const float u = h.nesterov ? fmaf(mu, mn, gv[e]) : mn;
+          mv[e] = mn;
+          cache[ch][e] = u;
+          ss = fmaf(u, u, ss);
+        }
+        store_m(mo, vec, ch, lane, cols, mv);
+      }
+    }
+    for (int ch = kProCachedChunks; ch < nch; ++ch) {
+      float gv[8], mv[8];
+      load_g_m(g, mo, vec, ch, lane, cols, gv, mv);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float mn = fmaf(mu, mv[e], gv[e]);
+        const float u = h.nesterov ? fmaf(mu, mn, gv[e]) : mn;
+        mv[e] = mn;
+        ss = fmaf(u, u, ss);
+      }
+      store_m(mo, vec, ch, lane, cols, mv);
+    }
+    ss = warp_allreduce_sum(ss);
+    const float inv = h.eq_r ? 1.f / (sqrtf(ss) + h.eps_row) : 1.f;
+    fro += ss * inv * inv;
+
+    // Pass 2: normalised row in bf16.
+#pragma unroll
+    for (int ch = 0; ch < kProCachedChunks; ++ch) {
+      if (ch < nch) {
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = cache[ch][e] * inv;
+        emit_x(xrow, srow, tr, vec, ch, lane, cols, x);
+      }
+    }
+    for (int ch = kProCachedChunks; ch < nch; ++ch) {
+      // Rows longer than the register cache: recompute U from G and the
+      // momentum this thread has just written.
+      float gv[8], mv[8], x[8];
+      load_g_m(g, mo, vec, ch, lane, cols, gv, mv);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float u = h.nesterov ? fmaf(mu, mv[e], gv[e]) : mv[e];
+        x[e] = u * inv;
+      }
+      emit_x(xrow, srow, tr, vec, ch, lane, cols, x);
+    }
+  }
+
+  if (lane == 0) warp_sums[warp] = fro;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kProThreads / 32; ++w) s += warp_sums[w];
+    partials[blockIdx.x] = s;
+  }
+
+  if (tr) {
+    // X[c][row0 + r] = stage[r][c]: 8 stored rows -> one 16-byte store.
+    const int ngrp = (it.nrows + 7) / 8;
+    __nv_bfloat16* xbase = md.x[0];
+    for (int idx = threadIdx.x; idx < cols * ngrp; idx += kProThreads) {
+      const int c = idx / ngrp;
+      const int grp = idx - c * ngrp;
+      const int r0 = grp * 8;
+      __nv_bfloat16* dst = xbase + static_cast<size_t>(c) * md.ldx + it.row0 + r0;
+      if (r0 + 8 <= it.nrows && ((it.row0 + r0) & 7) == 0) {
+        __align__(16) __nv_bfloat16 v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = stage[(r0 + k) * sld + c];
+        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(v);
+      } else {
+        for (int k = 0; k < 8 && r0 + k < it.nrows; ++k)
+          dst[k] = stage[(r0 + k) * sld + c];
+      }
+    }
+  }
+}
+
+// ns_steps == 0: O = s X~ straight from the prologue's output, then the
+// decoupled decay and scaled update.  One block per prologue work item.
+__global__ void __launch_bounds__(kProThreads)
+muon_final_noiter_kernel(const MatDev* __restrict__ mats,
+                         const ProItem* __restrict__ items,
+                         const float* __restrict__ partials, float lr, float wd,
+                         float eps_frob) {
+  const ProItem it = items[blockIdx.x];
+  const MatDev& md = mats[it.mat];
+  float sum = 0.f;
+  for (int i = 0; i < md.part_count; ++i) sum += partials[md.part_first + i];
+  const float s = 1.f / (sqrtf(sum) + eps_frob);
+  const float decay = 1.f - lr * wd;
+  const float step = lr * md.update_scale;
+  const int cols = md.cols;
+  const int total = it.nrows * cols;
+  for (int idx = threadIdx.x; idx < total; idx += kProThreads) {
+    const int r = it.row0 + idx / cols;
+    const int c = idx - (idx / cols) * cols;
+    const size_t xo = md.transposed
+                          ? static_cast<size_t>(c) * md.ldx + r
+                          : static_cast<size_t>(r) * md.ldx + c;
+    const float o = s * __bfloat162float(md.x[0][xo]);
+    const size_t wo = static_cast<size_t>(r) * cols + c;
+    md.w[wo] = fmaf(md.w[wo], decay, -step * o);
+    if (md.out) md.out[wo] = o;
+  }
+}
+
+}  // namespace muonb200

@@ -1,0 +1,638 @@
+// C ABI of the batched Muon step and the batched EMA (include/muon_b200.h):
+// argument validation, the plan (shapes -> workspace layout, work lists and
+// tile lists, built once), TMA descriptor encoding, and the launch sequence
+//
+//   prologue  ->  K x (gram -> poly -> apply)      (1 + 3K launches)
+//
+// on the caller's stream.  No device memory is allocated after
+// muon_plan_create.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "muon_b200.h"
+
+#include "k_ema.cuh"
+#include "k_ns_gemm.cuh"
+#include "k_prologue.cuh"
+#include "muon_types.cuh"
+
+using namespace muonb200;
+
+namespace {
+
+constexpr int kGramStages = 6;
+constexpr int kApplyStages = 4;
+using GramCfg = NsCfg<kGramN, false, kGramStages>;
+using ApplyCfg = NsCfg<kApplyN, true, kApplyStages>;
+constexpr int kMaxNsSteps = 16;
+constexpr int kMaxMats = 4096;
+constexpr int kMaxLaunchesPerStep = 1 + 3 * kMaxNsSteps;
+constexpr int kTimingSlots = 64;
+constexpr size_t kProSmemCap = 200 * 1024;
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
+                                  void*, const cuuint64_t*, const cuuint64_t*,
+                                  const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                         cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 matrix of `rows` x `cols` elements with leading dimension `ld`,
+// 128-byte swizzled boxes of box_cols x box_rows.
+bool encode_bf16_2d(CUtensorMap* tm, void* base, int rows, int cols, int ld,
+                    int box_cols, int box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols),
+                        static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols),
+                       static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Geom {
+  int rows, cols, m, n, ldx, lda, transposed;
+  size_t x_off[2], a_off, b_off;
+  int part_first, part_count;
+};
+
+struct TimingSlot {
+  cudaEvent_t ev[kMaxLaunchesPerStep + 1];
+  int kind[kMaxLaunchesPerStep];
+  int n = 0;
+  bool pending = false;
+};
+
+bool finite(float v) { return std::isfinite(v); }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+struct muon_plan {
+  int device = 0;
+  int num_sms = 148;
+  int n_mats = 0;
+  int max_ns = 0;
+  std::vector<Geom> geom;
+  std::vector<ProItem> items;
+  std::vector<NsTile> gram, poly, apply;
+  size_t ws_bytes = 0;
+  size_t part_off = 0;
+  size_t pro_smem = 0;
+
+  // device table: [MatDev x n_mats][ProItem][gram][poly][apply][err]
+  void* d_block = nullptr;
+  MatDev* d_mats = nullptr;
+  ProItem* d_items = nullptr;
+  NsTile* d_gram = nullptr;
+  NsTile* d_poly = nullptr;
+  NsTile* d_apply = nullptr;
+  int32_t* d_err = nullptr;
+
+  std::vector<MatDev> h_mats;     // what the device table holds now
+  bool h_valid = false;
+  void* enc_ws = nullptr;         // workspace the tensor maps were encoded for
+
+  int fault = 0;
+  bool timing = false;
+  std::vector<TimingSlot> slots;
+  int slot_head = 0;
+  double kind_ms[MUON_KIND_COUNT] = {};
+  long long kind_launches[MUON_KIND_COUNT] = {};
+};
+
+namespace {
+
+void harvest(muon_plan* plan, TimingSlot& s) {
+  if (!s.pending) return;
+  cudaEventSynchronize(s.ev[s.n]);
+  for (int i = 0; i < s.n; ++i) {
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, s.ev[i], s.ev[i + 1]) == cudaSuccess) {
+      plan->kind_ms[s.kind[i]] += ms;
+      plan->kind_launches[s.kind[i]] += 1;
+    }
+  }
+  s.pending = false;
+}
+
+struct Recorder {
+  muon_plan* plan;
+  cudaStream_t stream;
+  TimingSlot* slot = nullptr;
+  Recorder(muon_plan* p, cudaStream_t s) : plan(p), stream(s) {
+    if (!plan->timing) return;
+    slot = &plan->slots[plan->slot_head];
+    plan->slot_head = (plan->slot_head + 1) % kTimingSlots;
+    harvest(plan, *slot);
+    slot->n = 0;
+    cudaEventRecord(slot->ev[0], stream);
+  }
+  void after(int kind) {
+    if (!slot) return;
+    slot->kind[slot->n] = kind;
+    cudaEventRecord(slot->ev[slot->n + 1], stream);
+    slot->n += 1;
+  }
+  void finish() {
+    if (slot && slot->n > 0) slot->pending = true;
+  }
+};
+
+int pro_rows_per_item(int rows, int cols) {
+  if (rows <= cols) return kProRows;
+  size_t per_row = static_cast<size_t>(cols + 2) * 2;
+  int rt = static_cast<int>(std::min<size_t>(kProRows, kProSmemCap / per_row));
+  if (rt >= 8) rt &= ~7;
+  return std::max(rt, 1);
+}
+
+void sort_tiles(std::vector<NsTile>& v) {
+  std::stable_sort(v.begin(), v.end(),
+                   [](const NsTile& a, const NsTile& b) { return a.kt > b.kt; });
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t muon_abi_version(void) { return 100; }
+
+const char* muon_status_string(muon_status_t s) {
+  switch (s) {
+    case MUON_OK: return "ok";
+    case MUON_ERR_INVALID_ARG: return "invalid argument";
+    case MUON_ERR_UNSUPPORTED: return "unsupported shape or step count";
+    case MUON_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+    case MUON_ERR_CUDA: return "CUDA error";
+    case MUON_ERR_TIMEOUT: return "device-side wait timed out";
+    case MUON_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+  }
+  return "unknown status";
+}
+
+int32_t muon_step_launches(int32_t ns_steps) {
+  if (ns_steps < 0) return 0;
+  return ns_steps == 0 ? 2 : 1 + 3 * ns_steps;
+}
+
+int32_t ema_update_launches(int32_t n_tensors) {
+  return n_tensors <= 0 ? 0 : (n_tensors + kEmaMaxSegs - 1) / kEmaMaxSegs;
+}
+
+muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
+                               int32_t n_mats, int32_t max_ns_steps,
+                               muon_plan_t** out) {
+  if (!out) return MUON_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!rows || !cols || n_mats < 1 || n_mats > kMaxMats) return MUON_ERR_INVALID_ARG;
+  if (max_ns_steps < 0 || max_ns_steps > kMaxNsSteps) return MUON_ERR_UNSUPPORTED;
+  for (int i = 0; i < n_mats; ++i) {
+    if (rows[i] < 1 || cols[i] < 1) return MUON_ERR_INVALID_ARG;
+    // tile coordinates are 16-bit; keep every dimension well inside
+    if (rows[i] > (1 << 20) || cols[i] > (1 << 20)) return MUON_ERR_UNSUPPORTED;
+    if (static_cast<long long>(rows[i]) * cols[i] > (1ll << 31) - 1)
+      return MUON_ERR_UNSUPPORTED;
+  }
+
+  muon_plan* plan = new (std::nothrow) muon_plan();
+  if (!plan) return MUON_ERR_INVALID_ARG;
+  plan->n_mats = n_mats;
+  plan->max_ns = max_ns_steps;
+  if (cudaGetDevice(&plan->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&plan->num_sms, cudaDevAttrMultiProcessorCount,
+                             plan->device) != cudaSuccess) {
+    delete plan;
+    return MUON_ERR_CUDA;
+  }
+
+  // Geometry, workspace layout, prologue work items, tile lists.
+  size_t off = 0;
+  plan->geom.resize(n_mats);
+  for (int i = 0; i < n_mats; ++i) {
+    Geom& g = plan->geom[i];
+    g.rows = rows[i];
+    g.cols = cols[i];
+    g.transposed = rows[i] > cols[i];
+    g.m = std::min(rows[i], cols[i]);
+    g.n = std::max(rows[i], cols[i]);
+    g.ldx = static_cast<int>(align_up(g.n, 8));
+    g.lda = static_cast<int>(align_up(g.m, 8));
+    for (int b = 0; b < 2; ++b) {
+      g.x_off[b] = off;
+      off = align_up(off + static_cast<size_t>(g.m) * g.ldx * 2, 1024);
+    }
+    g.a_off = off;
+    off = align_up(off + static_cast<size_t>(g.m) * g.lda * 2, 1024);
+    g.b_off = off;
+    off = align_up(off + static_cast<size_t>(g.m) * g.lda * 2, 1024);
+
+    const int rt = pro_rows_per_item(g.rows, g.cols);
+    g.part_first = static_cast<int>(plan->items.size());
+    for (int r0 = 0; r0 < g.rows; r0 += rt) {
+      ProItem it{i, r0, std::min(rt, g.rows - r0), 0};
+      plan->items.push_back(it);
+    }
+    g.part_count = static_cast<int>(plan->items.size()) - g.part_first;
+    if (g.transposed)
+      plan->pro_smem = std::max(plan->pro_smem,
+                                static_cast<size_t>(rt) * (g.cols + 2) * 2);
+
+    const int tm = ceil_div(g.m, kTileM);
+    for (int ti = 0; ti < tm; ++ti)
+      for (int tj = ti; tj < tm; ++tj) {
+        plan->gram.push_back(NsTile{static_cast<uint16_t>(i), static_cast<uint16_t>(ti),
+                                    static_cast<uint16_t>(tj),
+                                    static_cast<uint16_t>(ceil_div(g.n, kTileK))});
+        plan->poly.push_back(NsTile{static_cast<uint16_t>(i), static_cast<uint16_t>(ti),
+                                    static_cast<uint16_t>(tj),
+                                    static_cast<uint16_t>(ceil_div(g.m, kTileK))});
+      }
+    const int tn = ceil_div(g.n, kApplyN);
+    for (int ti = 0; ti < tm; ++ti)
+      for (int tj = 0; tj < tn; ++tj)
+        plan->apply.push_back(NsTile{static_cast<uint16_t>(i), static_cast<uint16_t>(ti),
+                                     static_cast<uint16_t>(tj),
+                                     static_cast<uint16_t>(ceil_div(g.m, kTileK))});
+  }
+  if (plan->items.size() > 0x7FFFFFFF ||
+      plan->gram.size() > 0x7FFFFFFF || plan->apply.size() > 0x7FFFFFFF) {
+    delete plan;
+    return MUON_ERR_UNSUPPORTED;
+  }
+  sort_tiles(plan->gram);
+  sort_tiles(plan->poly);
+  sort_tiles(plan->apply);
+  plan->part_off = off;
+  off = align_up(off + plan->items.size() * sizeof(float), 1024);
+  plan->ws_bytes = off;
+
+  // Device table.
+  size_t t_off = 0;
+  const size_t mats_off = t_off;
+  t_off = align_up(t_off + sizeof(MatDev) * n_mats, 256);
+  const size_t items_off = t_off;
+  t_off = align_up(t_off + sizeof(ProItem) * plan->items.size(), 256);
+  const size_t gram_off = t_off;
+  t_off = align_up(t_off + sizeof(NsTile) * plan->gram.size(), 256);
+  const size_t poly_off = t_off;
+  t_off = align_up(t_off + sizeof(NsTile) * plan->poly.size(), 256);
+  const size_t apply_off = t_off;
+  t_off = align_up(t_off + sizeof(NsTile) * plan->apply.size(), 256);
+  const size_t err_off = t_off;
+  t_off += 256;
+  if (cudaMalloc(&plan->d_block, t_off) != cudaSuccess) {
+    cudaGetLastError();
+    delete plan;
+    return MUON_ERR_CUDA;
+  }
+  char* base = static_cast<char*>(plan->d_block);
+  plan->d_mats = reinterpret_cast<MatDev*>(base + mats_off);
+  plan->d_items = reinterpret_cast<ProItem*>(base + items_off);
+  plan->d_gram = reinterpret_cast<NsTile*>(base + gram_off);
+  plan->d_poly = reinterpret_cast<NsTile*>(base + poly_off);
+  plan->d_apply = reinterpret_cast<NsTile*>(base + apply_off);
+  plan->d_err = reinterpret_cast<int32_t*>(base + err_off);
+  bool ok =
+      cudaMemcpy(plan->d_items, plan->items.data(), sizeof(ProItem) * plan->items.size(),
+                 cudaMemcpyHostToDevice) == cudaSuccess &&
+      cudaMemcpy(plan->d_gram, plan->gram.data(), sizeof(NsTile) * plan->gram.size(),
+                 cudaMemcpyHostToDevice) == cudaSuccess &&
+      cudaMemcpy(plan->d_poly, plan->poly.data(), sizeof(NsTile) * plan->poly.size(),
+                 cudaMemcpyHostToDevice) == cudaSuccess &&
+      cudaMemcpy(plan->d_apply, plan->apply.data(), sizeof(NsTile) * plan->apply.size(),
+                 cudaMemcpyHostToDevice) == cudaSuccess &&
+      cudaMemset(plan->d_err, 0, sizeof(int32_t)) == cudaSuccess;
+  ok = ok &&
+       cudaFuncSetAttribute(ns_gemm_kernel<kGramN, false, kGramStages>,
+                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            static_cast<int>(GramCfg::kSmemBytes)) == cudaSuccess &&
+       cudaFuncSetAttribute(ns_gemm_kernel<kApplyN, true, kApplyStages>,
+                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            static_cast<int>(ApplyCfg::kSmemBytes)) == cudaSuccess &&
+       cudaFuncSetAttribute(muon_prologue_kernel,
+                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            static_cast<int>(std::max<size_t>(plan->pro_smem, 1024))) ==
+           cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    cudaFree(plan->d_block);
+    delete plan;
+    return MUON_ERR_CUDA;
+  }
+  plan->h_mats.resize(n_mats);
+  *out = plan;
+  return MUON_OK;
+}
+
+size_t muon_plan_workspace_bytes(const muon_plan_t* plan) {
+  return plan ? plan->ws_bytes : 0;
+}
+
+void muon_plan_destroy(muon_plan_t* plan) {
+  if (!plan) return;
+  cudaDeviceSynchronize();
+  for (auto& s : plan->slots)
+    for (auto& e : s.ev)
+      if (e) cudaEventDestroy(e);
+  if (plan->d_block) cudaFree(plan->d_block);
+  delete plan;
+}
+
+muon_status_t muon_plan_set_fault(muon_plan_t* plan, int32_t fault) {
+  if (!plan || fault < 0 || fault > 1) return MUON_ERR_INVALID_ARG;
+  plan->fault = fault;
+  return MUON_OK;
+}
+
+muon_status_t muon_plan_set_timing(muon_plan_t* plan, int32_t enable) {
+  if (!plan) return MUON_ERR_INVALID_ARG;
+  if (enable && plan->slots.empty()) {
+    plan->slots.resize(kTimingSlots);
+    for (auto& s : plan->slots)
+      for (auto& e : s.ev) {
+        e = nullptr;
+        if (cudaEventCreate(&e) != cudaSuccess) return MUON_ERR_CUDA;
+      }
+  }
+  plan->timing = enable != 0;
+  return MUON_OK;
+}
+
+muon_status_t muon_plan_timing_read(muon_plan_t* plan, int32_t* launches,
+                                    double* ms, int32_t n_kinds) {
+  if (!plan || n_kinds < 0) return MUON_ERR_INVALID_ARG;
+  // Harvest in issue order: oldest slot first.
+  for (int k = 0; k < static_cast<int>(plan->slots.size()); ++k)
+    harvest(plan, plan->slots[(plan->slot_head + k) % plan->slots.size()]);
+  for (int k = 0; k < n_kinds && k < MUON_KIND_COUNT; ++k) {
+    if (launches) launches[k] = static_cast<int32_t>(plan->kind_launches[k]);
+    if (ms) ms[k] = plan->kind_ms[k];
+  }
+  for (int k = 0; k < MUON_KIND_COUNT; ++k) {
+    plan->kind_ms[k] = 0.0;
+    plan->kind_launches[k] = 0;
+  }
+  return MUON_OK;
+}
+
+muon_status_t muon_get_last_error(muon_plan_t* plan, muon_stream_t stream) {
+  if (!plan) return MUON_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MUON_ERR_CUDA;
+  int32_t word = 0;
+  if (cudaMemcpy(&word, plan->d_err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  if (word != 0) {
+    cudaMemset(plan->d_err, 0, sizeof(int32_t));
+    cudaDeviceSynchronize();
+    return MUON_ERR_TIMEOUT;
+  }
+  if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
+  return MUON_OK;
+}
+
+muon_status_t muon_step_batched(muon_plan_t* plan, const muon_matrix_t* mats,
+                                const muon_hyper_t* hyper,
+                                const float* ns_coeffs, int32_t ns_steps,
+                                void* workspace, size_t workspace_bytes,
+                                muon_stream_t stream) {
+  // ---- validation (host, before anything is enqueued)
+  if (!plan || !mats || !hyper) return MUON_ERR_INVALID_ARG;
+  if (ns_steps < 0 || ns_steps > plan->max_ns) return MUON_ERR_UNSUPPORTED;
+  if (ns_steps > 0 && !ns_coeffs) return MUON_ERR_INVALID_ARG;
+  for (int k = 0; k < 3 * ns_steps; ++k)
+    if (!finite(ns_coeffs[k])) return MUON_ERR_INVALID_ARG;
+  const muon_hyper_t h = *hyper;
+  if (!finite(h.momentum) || !finite(h.lr) || !finite(h.weight_decay) ||
+      !finite(h.eps_row) || !finite(h.eps_frob) || h.eps_row < 0.f ||
+      h.eps_frob < 0.f || (h.nesterov != 0 && h.nesterov != 1) ||
+      (h.eq_r != 0 && h.eq_r != 1))
+    return MUON_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < plan->ws_bytes) return MUON_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MUON_ERR_WORKSPACE;
+  for (int i = 0; i < plan->n_mats; ++i) {
+    const muon_matrix_t& mt = mats[i];
+    const Geom& g = plan->geom[i];
+    if (mt.rows != g.rows || mt.cols != g.cols) return MUON_ERR_UNSUPPORTED;
+    if (!mt.w || !mt.momentum || !mt.grad_bf16) return MUON_ERR_INVALID_ARG;
+    if (!finite(mt.update_scale)) return MUON_ERR_INVALID_ARG;
+    if (!aligned16(mt.w) || !aligned16(mt.momentum) || !aligned16(mt.grad_bf16) ||
+        (mt.update_out && !aligned16(mt.update_out)))
+      return MUON_ERR_ALIGNMENT;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // ---- per-matrix device table (uploaded only when something changed)
+  char* ws = static_cast<char*>(workspace);
+  const bool reencode = plan->enc_ws != workspace;
+  std::vector<MatDev>& hm = plan->h_mats;
+  if (reencode) {
+    for (int i = 0; i < plan->n_mats; ++i) {
+      const Geom& g = plan->geom[i];
+      MatDev& d = hm[i];
+      std::memset(&d, 0, sizeof(MatDev));
+      for (int b = 0; b < 2; ++b) {
+        d.x[b] = reinterpret_cast<__nv_bfloat16*>(ws + g.x_off[b]);
+        if (!encode_bf16_2d(&d.tm_xk[b], d.x[b], g.m, g.n, g.ldx, kTileK, kTileM) ||
+            !encode_bf16_2d(&d.tm_xn[b], d.x[b], g.m, g.n, g.ldx, 64, kTileK)) {
+          plan->enc_ws = nullptr;
+          plan->h_valid = false;
+          return MUON_ERR_CUDA;
+        }
+      }
+      d.a = reinterpret_cast<__nv_bfloat16*>(ws + g.a_off);
+      d.b = reinterpret_cast<__nv_bfloat16*>(ws + g.b_off);
+      if (!encode_bf16_2d(&d.tm_a, d.a, g.m, g.m, g.lda, kTileK, kTileM) ||
+          !encode_bf16_2d(&d.tm_b, d.b, g.m, g.m, g.lda, kTileK, kTileM)) {
+        plan->enc_ws = nullptr;
+        plan->h_valid = false;
+        return MUON_ERR_CUDA;
+      }
+      d.rows = g.rows;
+      d.cols = g.cols;
+      d.m = g.m;
+      d.n = g.n;
+      d.ldx = g.ldx;
+      d.lda = g.lda;
+      d.transposed = g.transposed;
+      d.part_first = g.part_first;
+      d.part_count = g.part_count;
+    }
+    plan->enc_ws = workspace;
+    plan->h_valid = false;
+  }
+  bool changed = !plan->h_valid;
+  for (int i = 0; i < plan->n_mats; ++i) {
+    MatDev& d = hm[i];
+    const muon_matrix_t& mt = mats[i];
+    if (d.w != mt.w || d.mom != mt.momentum ||
+        d.g != mt.grad_bf16 || d.out != mt.update_out ||
+        std::memcmp(&d.update_scale, &mt.update_scale, sizeof(float)) != 0) {
+      d.w = mt.w;
+      d.mom = mt.momentum;
+      d.g = mt.grad_bf16;
+      d.out = mt.update_out;
+      d.update_scale = mt.update_scale;
+      changed = true;
+    }
+  }
+  if (changed) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return MUON_ERR_CUDA;
+    // A host-to-device table copy cannot be captured from pageable memory:
+    // run one call with the same buffers before capturing.
+    if (cap != cudaStreamCaptureStatusNone) return MUON_ERR_UNSUPPORTED;
+    // Pageable source: the call returns once the bytes are staged, so the
+    // host table may change right after; the copy is ordered on `st` after
+    // every earlier kernel of this plan.
+    if (cudaMemcpyAsync(plan->d_mats, hm.data(), sizeof(MatDev) * plan->n_mats,
+                        cudaMemcpyHostToDevice, st) != cudaSuccess) {
+      plan->h_valid = false;
+      return MUON_ERR_CUDA;
+    }
+    plan->h_valid = true;
+  }
+
+  // ---- launches
+  HyperDev hd{h.momentum, h.lr, h.weight_decay, h.eps_row, h.eps_frob,
+              h.nesterov, h.eq_r};
+  float* partials = reinterpret_cast<float*>(ws + plan->part_off);
+  Recorder rec(plan, st);
+
+  muon_prologue_kernel<<<static_cast<unsigned>(plan->items.size()), kProThreads,
+                         plan->pro_smem, st>>>(plan->d_mats, plan->d_items, hd,
+                                               partials);
+  rec.after(MUON_KIND_PROLOGUE);
+
+  if (ns_steps == 0) {
+    muon_final_noiter_kernel<<<static_cast<unsigned>(plan->items.size()),
+                               kProThreads, 0, st>>>(
+        plan->d_mats, plan->d_items, partials, h.lr, h.weight_decay, h.eps_frob);
+    rec.after(MUON_KIND_FINAL);
+  }
+  for (int k = 0; k < ns_steps; ++k) {
+    NsParams p{};
+    p.mats = plan->d_mats;
+    p.partials = partials;
+    p.err = plan->d_err;
+    p.src = k & 1;
+    p.fault = plan->fault;
+    p.fresh = changed ? 1 : 0;
+    p.a = ns_coeffs[3 * k + 0];
+    p.b = ns_coeffs[3 * k + 1];
+    p.c = ns_coeffs[3 * k + 2];
+    p.lr = h.lr;
+    p.wd = h.weight_decay;
+    p.eps_frob = h.eps_frob;
+
+    p.tiles = plan->d_gram;
+    p.n_tiles = static_cast<int>(plan->gram.size());
+    p.mode = kModeGram;
+    p.first = k == 0;
+    p.last = 0;
+    ns_gemm_kernel<kGramN, false, kGramStages>
+        <<<std::min(p.n_tiles, plan->num_sms), 192, GramCfg::kSmemBytes, st>>>(p);
+    rec.after(MUON_KIND_GRAM);
+
+    p.tiles = plan->d_poly;
+    p.n_tiles = static_cast<int>(plan->poly.size());
+    p.mode = kModePoly;
+    p.first = 0;
+    p.fault = 0;
+    ns_gemm_kernel<kGramN, false, kGramStages>
+        <<<std::min(p.n_tiles, plan->num_sms), 192, GramCfg::kSmemBytes, st>>>(p);
+    rec.after(MUON_KIND_POLY);
+
+    p.tiles = plan->d_apply;
+    p.n_tiles = static_cast<int>(plan->apply.size());
+    p.mode = kModeApply;
+    p.first = k == 0;
+    p.last = k == ns_steps - 1;
+    ns_gemm_kernel<kApplyN, true, kApplyStages>
+        <<<std::min(p.n_tiles, plan->num_sms), 192, ApplyCfg::kSmemBytes, st>>>(p);
+    rec.after(MUON_KIND_APPLY);
+  }
+  rec.finish();
+  if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
+  return MUON_OK;
+}
+
+muon_status_t ema_update_batched(float* const* ema, const float* const* params,
+                                 const int64_t* numel, int32_t n_tensors,
+                                 float decay, muon_stream_t stream) {
+  if (n_tensors < 0) return MUON_ERR_INVALID_ARG;
+  if (n_tensors == 0) return MUON_OK;
+  if (!ema || !params || !numel || !finite(decay)) return MUON_ERR_INVALID_ARG;
+  for (int i = 0; i < n_tensors; ++i) {
+    if (numel[i] < 0) return MUON_ERR_INVALID_ARG;
+    if (numel[i] == 0) continue;
+    if (!ema[i] || !params[i]) return MUON_ERR_INVALID_ARG;
+    if (((reinterpret_cast<uintptr_t>(ema[i]) |
+          reinterpret_cast<uintptr_t>(params[i])) & 3u) != 0)
+      return MUON_ERR_ALIGNMENT;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int sms = 148;
+  {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MUON_ERR_CUDA;
+  }
+  const double omd = 1.0 - static_cast<double>(decay);
+  for (int first = 0; first < n_tensors; first += kEmaMaxSegs) {
+    EmaParams p{};
+    p.d = decay;
+    p.one_minus_d = static_cast<float>(omd);
+    long long units = 0;
+    int ns = 0;
+    for (int i = first; i < std::min(n_tensors, first + kEmaMaxSegs); ++i, ++ns) {
+      p.seg[ns].e = ema[i];
+      p.seg[ns].p = params[i];
+      p.seg[ns].numel = numel[i];
+      p.seg[ns].ubeg = units;
+      units += (numel[i] + 3) / 4;
+    }
+    p.n_seg = ns;
+    p.total_units = units;
+    if (units == 0) continue;
+    const long long want = (units + kEmaThreads - 1) / kEmaThreads;
+    const unsigned grid = static_cast<unsigned>(std::min<long long>(want, 8ll * sms));
+    ema_update_kernel<<<grid, kEmaThreads, 0, st>>>(p);
+  }
+  if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
+  return MUON_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,85 @@
+// Device-side tables shared by the host launcher and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+namespace muonb200 {
+
+constexpr int kTileM = 128;       // UMMA M (rows of a tile)
+constexpr int kTileK = 64;        // K per pipeline stage (one 128-B swizzle row)
+constexpr int kGramN = 128;       // square tiles for the symmetric products
+constexpr int kApplyN = 256;      // wide tiles for X <- a X + B X
+constexpr int kProRows = 32;      // rows per prologue work item
+constexpr int kProThreads = 256;  // 8 warps
+constexpr int kProCachedChunks = 8;  // row chunks (of 256 elements) kept in
+                                     // registers: rows up to 2048 are read once
+
+// Per-matrix record.  Tensor maps first (64-byte aligned), pointers after.
+struct alignas(64) MatDev {
+  CUtensorMap tm_xk[2];  // X ping/pong as a K-major operand, box 64 x 128
+  CUtensorMap tm_xn[2];  // X ping/pong as an MN-major operand, box 64 x 64
+  CUtensorMap tm_a;      // A = X X^T (m x m), box 64 x 128
+  CUtensorMap tm_b;      // B = b A + c A A (m x m), box 64 x 128
+  __nv_bfloat16* x[2];   // m x ldx each
+  __nv_bfloat16* a;      // m x lda
+  __nv_bfloat16* b;      // m x lda
+  float* w;              // rows x cols (caller)
+  float* mom;            // rows x cols (caller)
+  const uint16_t* g;     // rows x cols bf16 bits (caller)
+  float* out;            // rows x cols or null (caller)
+  int32_t rows, cols;    // stored shape
+  int32_t m, n;          // working shape, m <= n
+  int32_t ldx, lda;      // leading dimensions (elements) of X and A/B
+  int32_t transposed;    // rows > cols
+  int32_t part_first;    // first prologue partial of this matrix
+  int32_t part_count;    // number of prologue partials
+  float update_scale;
+};
+
+// A prologue work item: up to kProRows stored rows of one matrix.
+struct ProItem {
+  int32_t mat;
+  int32_t row0;
+  int32_t nrows;
+  int32_t pad;
+};
+
+// A tile of one tensor-core phase.
+struct NsTile {
+  uint16_t mat;
+  uint16_t ti;   // tile row (128 rows)
+  uint16_t tj;   // tile column (128 or 256 columns)
+  uint16_t kt;   // number of 64-wide K blocks
+};
+
+struct HyperDev {
+  float mu, lr, wd, eps_row, eps_frob;
+  int32_t nesterov, eq_r;
+};
+
+enum NsMode : int32_t { kModeGram = 0, kModePoly = 1, kModeApply = 2 };
+
+struct NsParams {
+  const MatDev* mats;
+  const NsTile* tiles;
+  const float* partials;
+  int32_t* err;
+  int32_t n_tiles;
+  int32_t mode;
+  int32_t src;     // X buffer holding the current X
+  int32_t first;   // Newton-Schulz step 0: fold the Frobenius scale
+  int32_t last;    // last step: write W (and O) instead of X
+  int32_t fault;   // test hook (see muon_plan_set_fault)
+  int32_t fresh;   // the tensor maps were (re)written before this step
+  float a, b, c;
+  float lr, wd, eps_frob;
+};
+
+// Error word values (device -> host).
+constexpr int32_t kErrTimeoutProducer = 0x101;
+constexpr int32_t kErrTimeoutMma = 0x102;
+constexpr int32_t kErrTimeoutEpilogue = 0x103;
+
+}  // namespace muonb200

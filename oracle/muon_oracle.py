@@ -164,21 +164,24 @@ def newton_schulz(X: np.ndarray, coeffs: Sequence[Sequence[float]],
     input, so a fixed-coefficient schedule and a Polar-Express-style table are
     the same code path.  Each step is A = X X^T, B = b A + c A A, X <- a X + B X.
 
-    round_fn (diagnostic emulation only): applied where a bf16 path stores A,
-    B and the intermediate X.  The last X is not rounded.
+    round_fn (diagnostic emulation only): applied where a bf16 path stores
+    values.  Such a path stores A, then the matrix a I + B (so that
+    X <- (a I + B) X is one product; in exact arithmetic this is the same
+    step), then the intermediate X; the last X is not rounded.
     """
     X = np.asarray(X, dtype=np.float64)
     K = len(coeffs)
     for k, (a, b, c) in enumerate(coeffs):
         A = X @ X.T
-        if round_fn is not None:
+        if round_fn is None:
+            B = b * A + c * (A @ A)
+            X = a * X + B @ X
+        else:
             A = round_fn(A)
-        B = b * A + c * (A @ A)
-        if round_fn is not None:
-            B = round_fn(B)
-        X = a * X + B @ X
-        if round_fn is not None and k + 1 < K:
-            X = round_fn(X)
+            Bp = round_fn(a * np.eye(A.shape[0]) + b * A + c * (A @ A))
+            X = Bp @ X
+            if k + 1 < K:
+                X = round_fn(X)
     return X
 
 

@@ -80,14 +80,36 @@ def minimax_odd_quintic(lo: float, hi: float, iters: int = 100,
     return (float(coef[0]), float(coef[1]), float(coef[2])), float(E), xs
 
 
-def polar_express_table(steps: int = 4, lo: float = 1e-3, hi: float = 1.0):
-    """Greedy per-step minimax schedule: step k is optimal for the interval
-    left by steps 0..k-1.  Returns a list of (a, b, c) rows and the list of
-    intervals [lo_k, hi_k] each step starts from."""
-    rows, intervals = [], []
+def _image(coef, lo: float, hi: float) -> tuple[float, float]:
+    """Exact range of p over [lo, hi]: end points and interior critical
+    points."""
+    a, b, c = coef
+    xs = [lo, hi] + list(_interior_extrema(np.array(coef), lo, hi))
+    ys = [a * x + b * x ** 3 + c * x ** 5 for x in xs]
+    return min(ys), max(ys)
+
+
+def polar_express_table(steps: int = 4, lo: float = 1e-3, hi: float = 1.0,
+                        cushion: float = 0.0, inflate: float = 1.0):
+    """Greedy per-step minimax schedule.
+
+    Step k is the minimax odd quintic on the design interval
+    [max(lo_k, cushion * hi_k), inflate * hi_k]; the next interval
+    [lo_{k+1}, hi_{k+1}] is the exact image of [lo_k, hi_k] under it.
+    cushion > 0 keeps the design away from tiny lower ends (whose optimal
+    polynomials are steep, so bf16 rounding is amplified); inflate > 1 keeps
+    values slightly above the nominal upper end inside the region the
+    polynomial was designed for.  Both are stability margins of the same
+    kind the method uses; cushion = 0, inflate = 1 is the plain greedy
+    schedule.
+
+    Returns (rows of (a, b, c), nominal intervals, design intervals)."""
+    rows, intervals, design = [], [], []
     for _ in range(steps):
         intervals.append((lo, hi))
-        (a, b, c), E, _ = minimax_odd_quintic(lo, hi)
-        rows.append((a, b, c))
-        lo, hi = 1.0 - E, 1.0 + E
-    return rows, intervals
+        d_lo, d_hi = max(lo, cushion * hi), inflate * hi
+        design.append((d_lo, d_hi))
+        coef, _, _ = minimax_odd_quintic(d_lo, d_hi)
+        rows.append(coef)
+        lo, hi = _image(coef, lo, hi)
+    return rows, intervals, design

@@ -1,0 +1,118 @@
+"""Shared helpers of the GPU tests: seeded state on the device, one library
+step, and the fp64 oracle on the same inputs."""
+
+from __future__ import annotations
+
+import numpy as np
+
+import oracle.muon_oracle as mo
+from muon_optimizer_step_02_b200 import workloads as wl
+
+TOL_O = 2e-2        # relative Frobenius error of the bf16 Newton-Schulz output
+TOL_STATE = 1e-5    # fp32 momentum / EMA / weight states
+# Matrices with fewer than 16 rows or columns: each bf16 rounding of the few
+# entries of a I + B and X is not averaged out, about 2^-8 relative per step,
+# compounded over the steps by the polynomial's slope; the GPU path matches
+# the bf16-emulating oracle to 1e-2 there as well.
+TOL_O_TINY = 5e-2
+
+
+def tol_o(shape) -> float:
+    return TOL_O if min(shape) >= 16 else TOL_O_TINY
+
+
+def rel_fro(got, ref) -> float:
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = np.linalg.norm(ref)
+    num = np.linalg.norm(got - ref)
+    return float(num / den) if den > 0 else float(num)
+
+
+def oracle_hyper(h: wl.Hyper) -> mo.MuonHyper:
+    return mo.MuonHyper(momentum=h.momentum, lr=h.lr,
+                        weight_decay=h.weight_decay, eps_row=h.eps_row,
+                        eps_frob=h.eps_frob, nesterov=h.nesterov, eq_r=h.eq_r)
+
+
+class GpuMuon:
+    """Device state for one workload plus the library plan."""
+
+    def __init__(self, w: wl.Workload, seed: int = 1337, with_out=True):
+        import torch
+        from muon_optimizer_step_02_b200 import binding as B
+        self.w = w
+        self.seed = seed
+        self.plan = B.MuonPlan(w.shapes, max_ns_steps=max(len(w.coeffs), 1))
+        self.W = [torch.from_numpy(wl.weight(w, i, seed)).cuda()
+                  for i in range(w.n_mats)]
+        self.M = [torch.zeros_like(x) for x in self.W]
+        self.O = [torch.empty_like(x) for x in self.W] if with_out else None
+        self.ws = self.plan.alloc_workspace()
+        self.scales = wl.update_scales(w)
+
+    def grads(self, step: int):
+        import torch
+        return [torch.from_numpy(wl.grad_bits(self.w, i, step, self.seed)
+                                 .view(np.int16)).cuda().view(torch.bfloat16)
+                for i in range(self.w.n_mats)]
+
+    def step(self, G, coeffs=None):
+        self.plan.step(self.W, self.M, G, self.w.hyper,
+                       self.w.coeffs if coeffs is None else coeffs, self.ws,
+                       update_scales=self.scales, update_out=self.O)
+
+
+def check_step(g: GpuMuon, step: int, idx, coeffs=None, emu_tol=None,
+               report=None):
+    """Runs one library step and compares the listed matrices with the fp64
+    oracle applied to the same pre-step state.  Returns the worst errors."""
+    import torch
+    w = g.w
+    coeffs = w.coeffs if coeffs is None else coeffs
+    hyp = oracle_hyper(w.hyper)
+    W0 = {i: g.W[i].cpu().numpy().astype(np.float64) for i in idx}
+    M0 = {i: g.M[i].cpu().numpy().astype(np.float64) for i in idx}
+    G = g.grads(step)
+    Gh = {i: wl.bf16_bits_to_f32(wl.grad_bits(w, i, step, g.seed))
+          .astype(np.float64) for i in idx}
+    g.step(G, coeffs)
+    torch.cuda.synchronize()
+    assert g.plan.last_error() == 0
+    worst = {"O": 0.0, "M": 0.0, "W_given_O": 0.0, "W_e2e": 0.0,
+             "W_e2e_bound": 0.0, "O_emu": 0.0}
+    for i in idx:
+        W1 = g.W[i].cpu().numpy().astype(np.float64)
+        M1 = g.M[i].cpu().numpy().astype(np.float64)
+        O1 = g.O[i].cpu().numpy().astype(np.float64)
+        Wr, Mr, Or = mo.muon_step(W0[i], M0[i], Gh[i], hyp, coeffs,
+                                  g.scales[i])
+        e_o = rel_fro(O1, Or)
+        e_m = rel_fro(M1, Mr)
+        W_given = mo.decoupled_update(W0[i], O1, hyp.lr, hyp.weight_decay,
+                                      g.scales[i])
+        e_wg = rel_fro(W1, W_given)
+        e_we = rel_fro(W1, Wr)
+        # End-to-end weight error allowed by the update error alone.
+        bound = (hyp.lr * g.scales[i] * np.linalg.norm(O1 - Or)
+                 / max(np.linalg.norm(Wr), 1e-30)) + TOL_STATE
+        worst["O"] = max(worst["O"], e_o)
+        worst["M"] = max(worst["M"], e_m)
+        worst["W_given_O"] = max(worst["W_given_O"], e_wg)
+        worst["W_e2e"] = max(worst["W_e2e"], e_we)
+        worst["W_e2e_bound"] = max(worst["W_e2e_bound"], bound)
+        assert np.all(np.isfinite(O1)), f"matrix {i}: non-finite update"
+        assert e_o <= tol_o(w.shapes[i]), \
+            f"matrix {i} {w.shapes[i]}: O error {e_o:.3e}"
+        assert e_m <= TOL_STATE, f"matrix {i}: momentum error {e_m:.3e}"
+        assert e_wg <= TOL_STATE, f"matrix {i}: weight error {e_wg:.3e}"
+        assert e_we <= bound * 1.01, f"matrix {i}: e2e weight {e_we:.3e}"
+        if emu_tol is not None:
+            _, _, Oe = mo.muon_step(W0[i], M0[i], Gh[i], hyp, coeffs,
+                                    g.scales[i], emulate_bf16=True)
+            e_emu = rel_fro(O1, Oe)
+            worst["O_emu"] = max(worst["O_emu"], e_emu)
+            assert e_emu <= emu_tol, f"matrix {i}: vs bf16 emulation {e_emu:.3e}"
+    if report is not None:
+        report.append(worst)
+    return worst

@@ -172,37 +172,48 @@ def pin_ns_polar_factor(o):
 
 
 def pin_polar_express_table(o_pe):
-    """The generated Polar-Express-style table: each step equioscillates
-    (4 alternation points, the minimax certificate) on its interval, and
-    the composed schedule maps [lo0, 1] into the final band."""
+    """The generated Polar-Express-style table: each step equioscillates on
+    its design interval (4 alternation points: the minimax certificate), each
+    nominal interval is the image of the previous one, and the composed
+    schedule maps [lo0, 1] into the last image."""
     with open(os.path.join(HERE, "golden", "polar_express_k4.json")) as f:
         doc = json.load(f)
     rows, intervals = doc["coeffs"], doc["intervals"]
+    design = doc["design_intervals"]
     assert len(rows) == 4
-    for (a, b, c), (lo, hi) in zip(rows, intervals):
+    for (a, b, c), (lo, hi) in zip(rows, design):
         x = np.linspace(lo, hi, 400001)
         e = 1.0 - (a * x + b * x ** 3 + c * x ** 5)
         E = np.max(np.abs(e))
-        # alternation: sign changes between near-extremal points
         near = np.abs(np.abs(e) - E) < 1e-9 * max(1.0, E)
-        idx = np.flatnonzero(near)
-        signs = np.sign(e[idx])
+        signs = np.sign(e[np.flatnonzero(near)])
         alternations = 1 + int(np.sum(signs[1:] != signs[:-1]))
         assert alternations >= 4, (alternations, lo, hi)
         assert abs(e[0] - E) < 1e-9 and abs(e[-1] + E) < 1e-9
-    # Regenerating gives the stored numbers.
-    rows2, iv2 = o_pe.polar_express_table(4, *doc["initial_interval"])
+    for k in range(3):
+        a, b, c = rows[k]
+        lo, hi = intervals[k]
+        x = np.linspace(lo, hi, 400001)
+        y = a * x + b * x ** 3 + c * x ** 5
+        assert abs(y.min() - intervals[k + 1][0]) < 1e-8
+        assert abs(y.max() - intervals[k + 1][1]) < 1e-8
+    rows2, iv2, d2 = o_pe.polar_express_table(
+        4, *doc["initial_interval"], doc["cushion"], doc["inflate"])
     assert np.allclose(np.array(rows2), np.array(rows), rtol=1e-12)
     assert np.allclose(np.array(iv2), np.array(intervals), rtol=1e-12)
-    # The composed map sends [lo0, 1] into [1 - E4, 1 + E4].
+    assert np.allclose(np.array(d2), np.array(design), rtol=1e-12)
     lo0, hi0 = doc["initial_interval"]
     x = np.geomspace(lo0, hi0, 20001)
     y = _scalar_poly_chain(x, rows)
     a, b, c = rows[-1]
     lo3, hi3 = intervals[-1]
-    g = np.linspace(lo3, hi3, 200001)
-    E4 = np.max(np.abs(1 - (a * g + b * g ** 3 + c * g ** 5)))
-    assert y.min() >= 1 - E4 - 1e-9 and y.max() <= 1 + E4 + 1e-9
+    g = np.linspace(lo3, hi3, 400001)
+    p = a * g + b * g ** 3 + c * g ** 5
+    assert y.min() >= p.min() - 1e-9 and y.max() <= p.max() + 1e-9
+    # the plain greedy schedule (no margins) is a minimax chain too
+    r0, iv0, _ = o_pe.polar_express_table(2, 1e-3, 1.0)
+    (a, b, c) = r0[0]
+    assert abs((a * 1e-3 + b * 1e-9 + c * 1e-15) - iv0[1][0]) < 1e-12
 
 
 def pin_ns_equivariance(o):

@@ -1,0 +1,95 @@
+"""GPU vs fp64 oracle on the five workloads, through the C ABI.
+
+Tolerances: relative Frobenius error <= 2e-2 for the bf16 Newton-Schulz
+output O; <= 1e-5 for the fp32 momentum, for the weight given the library's
+O, and for the EMA; the end-to-end weight error must stay inside the bound
+implied by the O error.  Three consecutive steps with fresh gradients, so
+the momentum term is exercised with a non-zero buffer.
+"""
+import numpy as np
+import pytest
+
+import oracle.muon_oracle as mo
+from gpu_harness import GpuMuon, TOL_STATE, check_step, rel_fro
+from muon_optimizer_step_02_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+# Tight diagnostic: the same rounding points as the bf16 path.
+EMU_TOL = 1e-2
+
+
+def test_single_128():
+    w = wl.workload(1)
+    g = GpuMuon(w)
+    for step in range(3):
+        check_step(g, step, [0], emu_tol=EMU_TOL)
+
+
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_gpt11_all_matrices(cfg):
+    w = wl.workload(cfg)
+    g = GpuMuon(w)
+    rep = []
+    for step in range(3):
+        check_step(g, step, list(range(w.n_mats)), emu_tol=EMU_TOL, report=rep)
+    print(cfg, rep)
+
+
+def _sample(w, extra, seed=7):
+    first = {}
+    for i, s in enumerate(w.shapes):
+        first.setdefault(s, i)
+    rng = np.random.default_rng(seed)
+    more = rng.choice(w.n_mats, size=extra, replace=False).tolist()
+    return sorted(set(first.values()) | set(more))
+
+
+def test_gpt16_sampled():
+    w = wl.workload(4)
+    g = GpuMuon(w)
+    idx = _sample(w, 2)
+    check_step(g, 0, [idx[0]])
+    check_step(g, 1, idx, emu_tol=EMU_TOL)
+
+
+@pytest.mark.slow
+def test_gpt24_sampled():
+    w = wl.workload(5)
+    g = GpuMuon(w)
+    idx = _sample(w, 1)
+    check_step(g, 0, [])
+    check_step(g, 1, idx)
+
+
+def _ema_check(w, idx_check):
+    import torch
+    from muon_optimizer_step_02_b200 import binding as B
+    E, P, E0, P0 = [], [], {}, {}
+    for i in range(len(w.ema_numels())):
+        e, p = wl.ema_pair(w, i)
+        if i in idx_check:
+            E0[i], P0[i] = e.astype(np.float64), p.astype(np.float64)
+        E.append(torch.from_numpy(e).cuda())
+        P.append(torch.from_numpy(p).cuda())
+    B.ema_update_batched(E, P, w.ema_decay)
+    torch.cuda.synchronize()
+    worst = 0.0
+    for i in idx_check:
+        ref = mo.ema_update(E0[i], P0[i], w.ema_decay)
+        err = rel_fro(E[i].cpu().numpy(), ref)
+        worst = max(worst, err)
+        assert err <= TOL_STATE, (i, err)
+    return worst
+
+
+def test_ema_gpt11_all_tensors():
+    w = wl.workload(3)
+    _ema_check(w, set(range(len(w.ema_numels()))))
+
+
+@pytest.mark.slow
+def test_ema_gpt24_sampled():
+    w = wl.workload(5)
+    n = len(w.ema_numels())
+    _ema_check(w, {0, 5, 143, 144, 145, n - 1})
