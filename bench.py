@@ -23,7 +23,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -54,59 +53,71 @@ def load_peaks():
 # clocks
 # --------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
-              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    """Samples SM clock and clock-event reasons of this process's GPU every
+    few milliseconds (NVML, read-only) while the timed region runs."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, cuda_index: int, period_s: float = 0.005):
+        self.cuda_index = cuda_index
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = None
+        self._thread = None
+
+    def _handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.cuda_index).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            return pynvml.nvmlDeviceGetHandleByUUID(uuid)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.cuda_index)
 
     def start(self):
+        import threading
         try:
-            self.path = f"/tmp/muonb200_clocks_{os.getpid()}.csv"
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200",
-                 "-i", str(self.gpu)], stdout=self.fh,
-                stderr=subprocess.DEVNULL)
+            import pynvml
+            h = self._handle()
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(
+                h, pynvml.NVML_CLOCK_SM)
         except Exception:
-            self.proc = None
+            return
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(pynvml.nvmlDeviceGetClockInfo(
+                        h, pynvml.NVML_CLOCK_SM))
+                    self.reasons |= int(
+                        pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))
+                except Exception:
+                    pass
+                self._stop.wait(self.period)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self._thread is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.fh.close()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
-                 "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    smax.append(float(parts[2]))
-                except ValueError:
-                    continue
-                for name, val in zip(names, parts[5:9]):
-                    if val.lower().startswith("active"):
-                        reasons.add(name)
-        os.remove(self.path)
-        if not sm:
+        self._stop.set()
+        self._thread.join(timeout=2)
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(self.samples),
+                "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(k for k, bit in self.REASONS.items()
+                                  if self.reasons & bit),
+                "samples": len(self.samples), "source": "nvml"}
 
 
 # --------------------------------------------------------------------------
@@ -140,11 +151,17 @@ class Workload:
         self.P = [x.view(-1) for x in self.W] + self.extra
         self.E = [e.view(-1) for e in self.E]
 
+        # Arguments are marshalled once; a step only enqueues the launches.
+        self._muon = self.plan.bind(self.W, self.M, self.G, self.w.hyper,
+                                    self.w.coeffs, self.ws,
+                                    update_scales=self.scales)
+        self._ema = (B.ema_bind(self.E, self.P, self.w.ema_decay)
+                     if self.w.ema_decay is not None else None)
+
     def step(self):
-        self.plan.step(self.W, self.M, self.G, self.w.hyper, self.w.coeffs,
-                       self.ws, update_scales=self.scales)
-        if self.w.ema_decay is not None:
-            self.B.ema_update_batched(self.E, self.P, self.w.ema_decay)
+        self._muon()
+        if self._ema is not None:
+            self._ema()
 
     def launches_per_step(self) -> int:
         n = self.B.step_launches(len(self.w.coeffs))
@@ -216,7 +233,7 @@ def run_ours(args, rank, world, local_rank):
         reps = max(3, args.steps // 4)
         e0.record(stream)
         for _ in range(reps):
-            rep.B.ema_update_batched(rep.E, rep.P, w.ema_decay)
+            rep._ema()
         e1.record(stream)
         torch.cuda.synchronize()
         ema_ms = e0.elapsed_time(e1) / reps

@@ -158,6 +158,15 @@ class MuonPlan:
         CUDA tensors (updated in place); grads: bf16 CUDA tensors; hyper: an
         object with momentum, lr, weight_decay, eps_row, eps_frob, nesterov,
         eq_r; coeffs: ns_steps rows of (a, b, c)."""
+        self.bind(weights, momenta, grads, hyper, coeffs, workspace,
+                  update_scales, update_out)(stream)
+
+    def bind(self, weights, momenta, grads, hyper, coeffs, workspace,
+             update_scales: Optional[Sequence[float]] = None,
+             update_out=None):
+        """Checks and marshals the arguments once; returns a callable
+        `run(stream=None)` that enqueues muon_step_batched with them.  The
+        tensors must stay alive and in place while the callable is used."""
         import torch
         n = len(self.shapes)
         if not (len(weights) == len(momenta) == len(grads) == n):
@@ -189,11 +198,16 @@ class MuonPlan:
         carr = (c_float * max(len(flat), 1))(*flat)
         _check_tensor(workspace, torch.uint8, (workspace.numel(),),
                       "workspace")
-        st = lib().muon_step_batched(self._h, mats, ctypes.byref(hp), carr, k,
-                                     workspace.data_ptr(),
-                                     workspace.numel(),
-                                     _stream_handle(stream))
-        _check(st, "muon_step_batched")
+        fn = lib().muon_step_batched
+        h, hp_ref = self._h, ctypes.byref(hp)
+        ws_ptr, ws_n = workspace.data_ptr(), workspace.numel()
+        keep = (mats, hp, carr, weights, momenta, grads, update_out, workspace)
+
+        def run(stream=None):
+            _ = keep
+            _check(fn(h, mats, hp_ref, carr, k, ws_ptr, ws_n,
+                      _stream_handle(stream)), "muon_step_batched")
+        return run
 
     def last_error(self, stream=None) -> int:
         return int(lib().muon_get_last_error(self._h, _stream_handle(stream)))
@@ -235,6 +249,12 @@ def ema_update_batched(emas: Sequence, params: Sequence, decay: float,
                        stream=None):
     """E <- decay E + (1 - decay) P for every (E, P) pair (fp32 CUDA
     tensors, contiguous, same numel)."""
+    ema_bind(emas, params, decay)(stream)
+
+
+def ema_bind(emas: Sequence, params: Sequence, decay: float):
+    """Checks and marshals the arguments of ema_update_batched once; returns
+    a callable `run(stream=None)`."""
     import torch
     n = len(emas)
     if len(params) != n:
@@ -254,9 +274,15 @@ def ema_update_batched(emas: Sequence, params: Sequence, decay: float,
         e_arr[i] = e.data_ptr()
         p_arr[i] = p.data_ptr()
         num[i] = e.numel()
-    st = lib().ema_update_batched(e_arr, p_arr, num, n, float(decay),
-                                  _stream_handle(stream))
-    _check(st, "ema_update_batched")
+    fn = lib().ema_update_batched
+    keep = (e_arr, p_arr, num, list(emas), list(params))
+    d = float(decay)
+
+    def run(stream=None):
+        _ = keep
+        _check(fn(e_arr, p_arr, num, n, d, _stream_handle(stream)),
+               "ema_update_batched")
+    return run
 
 
 def step_launches(ns_steps: int) -> int:

@@ -1,8 +1,9 @@
 // K-EMA: E <- d E + (1 - d) P over many parameter tensors in one launch.
 //
 // The tensors form one flat space of 4-element units; each thread walks it
-// with a grid stride and keeps a cursor into the (monotonic) segment table,
-// so a warp almost always works inside one tensor.  16-byte aligned tensors
+// with a grid stride, finds its first tensor by binary search in the segment
+// table and then advances a cursor (units only increase), so a warp almost
+// always works inside one tensor.  16-byte aligned tensors
 // move as float4 (128-bit loads/stores); tails and unaligned tensors use
 // scalar accesses.
 //
@@ -16,7 +17,7 @@
 
 namespace muonb200 {
 
-constexpr int kEmaMaxSegs = 96;
+constexpr int kEmaMaxSegs = 320;  // 10 KB of kernel parameters
 constexpr int kEmaThreads = 256;
 
 struct EmaSeg {
@@ -37,9 +38,15 @@ struct EmaParams {
 __global__ void __launch_bounds__(kEmaThreads)
 ema_update_kernel(const __grid_constant__ EmaParams p) {
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  int cur = 0;
-  for (long long u = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-       u < p.total_units; u += stride) {
+  const long long u0 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  // last segment with ubeg <= u0
+  int lo = 0, hi = p.n_seg - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.seg[mid].ubeg <= u0) lo = mid; else hi = mid - 1;
+  }
+  int cur = lo;
+  for (long long u = u0; u < p.total_units; u += stride) {
     while (cur + 1 < p.n_seg && u >= p.seg[cur + 1].ubeg) ++cur;
     float* e = p.seg[cur].e;
     const float* q = p.seg[cur].p;

@@ -12,9 +12,9 @@
 // s = 1 / (||X~||_F + eps_frob) on the first step (the Frobenius
 // normalisation folded into the products), 1 afterwards.
 //
-// Roles (192 threads): warp 0 issues TMA loads into a ring of shared-memory
+// Roles (320 threads): warp 0 issues TMA loads into a ring of shared-memory
 // stages; warp 1 owns TMEM and issues tcgen05.mma (M = 128, N = BN, K = 16)
-// from one thread; warps 2-5 drain the double-buffered TMEM accumulator and
+// from one thread; warps 2-9 drain the double-buffered TMEM accumulator and
 // run the fused epilogue.  Every wait is bounded (see mbar_wait_bounded).
 //
 // Source of the step: PR #1396 "Record: Combined 3-Layer Recurrence +
@@ -31,6 +31,10 @@
 
 namespace muonb200 {
 
+constexpr int kEpiWarps = 8;                 // two per TMEM lane quadrant
+constexpr int kNsThreads = 64 + 32 * kEpiWarps;
+constexpr int kXposeLd = 34;                 // bf16 per row of a 32x32 block
+
 template <int BN, bool kBmn, int kStages>
 struct NsCfg {
   static constexpr int kABytes = kTileM * kTileK * 2;
@@ -38,8 +42,11 @@ struct NsCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kNumBars = 2 * kStages + 5;
-  static constexpr size_t kSmemBytes =
-      1024 + static_cast<size_t>(kStages) * kStageBytes + kNumBars * 8 + 16;
+  // per epilogue warp: a 32 x 32 bf16 block for the mirrored store
+  static constexpr int kXposeBytes = kBmn ? 0 : kEpiWarps * 32 * kXposeLd * 2;
+  static constexpr size_t kSmemBytes = 1024 +
+      static_cast<size_t>(kStages) * kStageBytes + kXposeBytes +
+      kNumBars * 8 + 16;
   static_assert(kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -102,26 +109,50 @@ __device__ __forceinline__ void store_row32_bf16(__nv_bfloat16* dst, int col0,
   }
 }
 
-// Column `row` of the mirrored tile: element (row, col0+e) goes to
-// (col0+e, row).  Lanes hold consecutive rows, so each store is coalesced
-// across the warp.
-__device__ __forceinline__ void store_col32_bf16(__nv_bfloat16* base, int ld,
-                                                 int row, int col0, int limit,
-                                                 const float (&v)[32]) {
+// The mirrored 32 x 32 block: lane l holds row (row0 + l), columns
+// col0..col0+31; the block is transposed through `buf` (per warp, 32 rows of
+// kXposeLd bf16) and lane l then writes row (col0 + l) of the mirror,
+// columns row0..row0+31, as four 16-byte stores.
+__device__ __forceinline__ void store_mirror32_bf16(__nv_bfloat16* base, int ld,
+                                                    int row0, int col0,
+                                                    int limit, int lane,
+                                                    __nv_bfloat16* buf,
+                                                    const float (&v)[32]) {
+  __nv_bfloat162* wrow = reinterpret_cast<__nv_bfloat162*>(buf + lane * kXposeLd);
 #pragma unroll
-  for (int e = 0; e < 32; ++e)
-    if (col0 + e < limit)
-      base[static_cast<size_t>(col0 + e) * ld + row] = __float2bfloat16_rn(v[e]);
+  for (int i = 0; i < 16; ++i)
+    wrow[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  __syncwarp();
+  const int mrow = col0 + lane;
+  if (mrow < limit) {
+    __nv_bfloat16* dst = base + static_cast<size_t>(mrow) * ld + row0;
+    if (row0 + 32 <= limit) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        __align__(16) __nv_bfloat16 h[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) h[k] = buf[(8 * q + k) * kXposeLd + lane];
+        reinterpret_cast<uint4*>(dst)[q] = *reinterpret_cast<uint4*>(h);
+      }
+    } else {
+      for (int k = 0; k < 32 && row0 + k < limit; ++k)
+        dst[k] = buf[k * kXposeLd + lane];
+    }
+  }
+  __syncwarp();
 }
 
 template <int BN, bool kBmn, int kStages>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kNsThreads, 1)
 ns_gemm_kernel(const __grid_constant__ NsParams p) {
   using Cfg = NsCfg<BN, kBmn, kStages>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * Cfg::kStageBytes);
+  __nv_bfloat16* xpose =
+      reinterpret_cast<__nv_bfloat16*>(smem + kStages * Cfg::kStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      smem + kStages * Cfg::kStageBytes + Cfg::kXposeBytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -144,7 +175,7 @@ ns_gemm_kernel(const __grid_constant__ NsParams p) {
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 128);
+      mbar_init(tempty_bar(a), 32 * kEpiWarps);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -260,8 +291,14 @@ ns_gemm_kernel(const __grid_constant__ NsParams p) {
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Eight warps: two per TMEM lane quadrant, splitting a tile's 32-column
+    // chunks between them.  Inputs of a chunk (A for poly, W for the update)
+    // are loaded before the accumulator so their latency overlaps.
+    const int ew = warp - 2;
     const int quad = warp & 3;             // TMEM lane quadrant of this warp
+    const int half = ew >> 2;              // chunk parity handled by this warp
     const int r_in = quad * 32 + lane;     // accumulator row of this thread
+    __nv_bfloat16* xbuf = xpose + ew * 32 * kXposeLd;
     int lt = 0;
     for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++lt) {
       const NsTile tl = p.tiles[t];
@@ -275,7 +312,8 @@ ns_gemm_kernel(const __grid_constant__ NsParams p) {
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      const int row = tl.ti * kTileM + r_in;
+      const int row0 = tl.ti * kTileM + quad * 32;
+      const int row = row0 + lane;
       const int m = md->m;
       const bool row_ok = row < m;
       const float s = p.first ? frob_scale(md, p.partials, p.eps_frob) : 1.f;
@@ -284,17 +322,18 @@ ns_gemm_kernel(const __grid_constant__ NsParams p) {
         __nv_bfloat16* outp = (p.mode == kModeGram) ? md->a : md->b;
         const bool mirror = tl.ti != tl.tj;
 #pragma unroll 1
-        for (int cc = 0; cc < BN / 32; ++cc) {
+        for (int cc = half; cc < BN / 32; cc += 2) {
+          const int col0 = tl.tj * BN + cc * 32;
+          float av[32];
+          if (p.mode == kModePoly && row_ok)
+            load_row32_bf16(md->a + static_cast<size_t>(row) * md->lda, col0, m, av);
           float v[32];
           tmem_load_32cols(tbase + cc * 32, v);
-          const int col0 = tl.tj * BN + cc * 32;
           if (p.mode == kModeGram) {
             const float s2 = s * s;
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] *= s2;
           } else if (row_ok) {
-            float av[32];
-            load_row32_bf16(md->a + static_cast<size_t>(row) * md->lda, col0, m, av);
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = fmaf(p.b, av[e], p.c * v[e]);
             if (!mirror && (r_in >> 5) == cc) {  // this row's diagonal element
@@ -304,66 +343,88 @@ ns_gemm_kernel(const __grid_constant__ NsParams p) {
                 if (e == d) v[e] += p.a;
             }
           }
-          if (row_ok) {
+          if (row_ok)
             store_row32_bf16(outp + static_cast<size_t>(row) * md->lda, col0, m, v);
-            if (mirror) store_col32_bf16(outp, md->lda, row, col0, m, v);
-          }
+          if (mirror)
+            store_mirror32_bf16(outp, md->lda, row0, col0, m, lane, xbuf, v);
         }
       } else {
         const int n = md->n;
         __nv_bfloat16* xd = md->x[p.src ^ 1] + static_cast<size_t>(row) * md->ldx;
         const float decay = 1.f - p.lr * p.wd;
         const float step = p.lr * md->update_scale;
+        const bool tr = md->transposed != 0;
 #pragma unroll 1
-        for (int cc = 0; cc < BN / 32; ++cc) {
+        for (int cc = half; cc < BN / 32; cc += 2) {
+          const int col0 = tl.tj * BN + cc * 32;
+          const bool live = row_ok && col0 < n;
+          // W (and only W) is read in the last step: all 32 loads first.
+          float wv[32];
+          float* w_row = nullptr;
+          const bool wvec = !tr && col0 + 32 <= n && (n & 3) == 0;
+          if (p.last && live) {
+            if (!tr) {
+              w_row = md->w + static_cast<size_t>(row) * n + col0;
+              if (wvec) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                  const float4 w4 = reinterpret_cast<const float4*>(w_row)[q];
+                  wv[4 * q] = w4.x; wv[4 * q + 1] = w4.y;
+                  wv[4 * q + 2] = w4.z; wv[4 * q + 3] = w4.w;
+                }
+              } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) wv[e] = col0 + e < n ? w_row[e] : 0.f;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                wv[e] = col0 + e < n
+                            ? md->w[static_cast<size_t>(col0 + e) * m + row] : 0.f;
+            }
+          }
           float v[32];
           tmem_load_32cols(tbase + cc * 32, v);
-          const int col0 = tl.tj * BN + cc * 32;
-          if (!row_ok || col0 >= n) continue;
+          if (!live) continue;
           if (p.first) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] *= s;
           }
           if (!p.last) {
             store_row32_bf16(xd, col0, n, v);
-          } else if (!md->transposed) {
-            // O (rows x cols) = X: this thread owns a contiguous row segment.
-            float* w = md->w + static_cast<size_t>(row) * n;
-            float* o = md->out ? md->out + static_cast<size_t>(row) * n : nullptr;
-            if (col0 + 32 <= n && (n & 3) == 0) {
+            continue;
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) wv[e] = fmaf(wv[e], decay, -step * v[e]);
+          if (!tr) {
+            float* o = md->out ? md->out + static_cast<size_t>(row) * n + col0 : nullptr;
+            if (wvec) {
 #pragma unroll
               for (int q = 0; q < 8; ++q) {
-                float4 wv = *reinterpret_cast<const float4*>(w + col0 + 4 * q);
-                wv.x = fmaf(wv.x, decay, -step * v[4 * q + 0]);
-                wv.y = fmaf(wv.y, decay, -step * v[4 * q + 1]);
-                wv.z = fmaf(wv.z, decay, -step * v[4 * q + 2]);
-                wv.w = fmaf(wv.w, decay, -step * v[4 * q + 3]);
-                *reinterpret_cast<float4*>(w + col0 + 4 * q) = wv;
+                reinterpret_cast<float4*>(w_row)[q] =
+                    make_float4(wv[4 * q], wv[4 * q + 1], wv[4 * q + 2], wv[4 * q + 3]);
                 if (o)
-                  *reinterpret_cast<float4*>(o + col0 + 4 * q) =
+                  reinterpret_cast<float4*>(o)[q] =
                       make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
               }
             } else {
 #pragma unroll
-              for (int e = 0; e < 32; ++e) {
+              for (int e = 0; e < 32; ++e)
                 if (col0 + e < n) {
-                  w[col0 + e] = fmaf(w[col0 + e], decay, -step * v[e]);
-                  if (o) o[col0 + e] = v[e];
+                  w_row[e] = wv[e];
+                  if (o) o[e] = v[e];
                 }
-              }
             }
           } else {
-            // O = X^T: W is n x m; element (row, col) of X lands at
-            // W[col][row], consecutive across the warp's lanes.
+            // O = X^T: element (row, col) of X lands at W[col][row];
+            // consecutive lanes write consecutive addresses.
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int col = col0 + e;
-              if (col < n) {
-                const size_t off = static_cast<size_t>(col) * m + row;
-                md->w[off] = fmaf(md->w[off], decay, -step * v[e]);
+            for (int e = 0; e < 32; ++e)
+              if (col0 + e < n) {
+                const size_t off = static_cast<size_t>(col0 + e) * m + row;
+                md->w[off] = wv[e];
                 if (md->out) md->out[off] = v[e];
               }
-            }
           }
         }
       }

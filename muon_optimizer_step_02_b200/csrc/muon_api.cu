@@ -182,6 +182,149 @@ void sort_tiles(std::vector<NsTile>& v) {
                    [](const NsTile& a, const NsTile& b) { return a.kt > b.kt; });
 }
 
+// Everything the launch sequence needs: where the device tables are.
+struct LaunchTables {
+  const MatDev* mats;
+  const ProItem* items;
+  int n_items;
+  const NsTile* gram;
+  int n_gram;
+  const NsTile* poly;
+  int n_poly;
+  const NsTile* apply;
+  int n_apply;
+  int32_t* err;
+  int num_sms;
+  size_t pro_smem;
+};
+
+muon_status_t validate_hyper(const muon_hyper_t* hyper, const float* ns_coeffs,
+                             int32_t ns_steps, int32_t max_ns) {
+  if (!hyper) return MUON_ERR_INVALID_ARG;
+  if (ns_steps < 0 || ns_steps > max_ns) return MUON_ERR_UNSUPPORTED;
+  if (ns_steps > 0 && !ns_coeffs) return MUON_ERR_INVALID_ARG;
+  for (int k = 0; k < 3 * ns_steps; ++k)
+    if (!finite(ns_coeffs[k])) return MUON_ERR_INVALID_ARG;
+  const muon_hyper_t& h = *hyper;
+  if (!finite(h.momentum) || !finite(h.lr) || !finite(h.weight_decay) ||
+      !finite(h.eps_row) || !finite(h.eps_frob) || h.eps_row < 0.f ||
+      h.eps_frob < 0.f || (h.nesterov != 0 && h.nesterov != 1) ||
+      (h.eq_r != 0 && h.eq_r != 1))
+    return MUON_ERR_INVALID_ARG;
+  return MUON_OK;
+}
+
+muon_status_t validate_matrix(const muon_matrix_t& mt, const Geom& g) {
+  if (mt.rows != g.rows || mt.cols != g.cols) return MUON_ERR_UNSUPPORTED;
+  if (!mt.w || !mt.momentum || !mt.grad_bf16) return MUON_ERR_INVALID_ARG;
+  if (!finite(mt.update_scale)) return MUON_ERR_INVALID_ARG;
+  if (!aligned16(mt.w) || !aligned16(mt.momentum) || !aligned16(mt.grad_bf16) ||
+      (mt.update_out && !aligned16(mt.update_out)))
+    return MUON_ERR_ALIGNMENT;
+  return MUON_OK;
+}
+
+// Workspace-dependent part of a matrix record: buffer pointers, tensor maps,
+// geometry.
+bool fill_workspace_fields(MatDev& d, const Geom& g, char* ws) {
+  std::memset(&d, 0, sizeof(MatDev));
+  for (int b = 0; b < 2; ++b) {
+    d.x[b] = reinterpret_cast<__nv_bfloat16*>(ws + g.x_off[b]);
+    if (!encode_bf16_2d(&d.tm_xk[b], d.x[b], g.m, g.n, g.ldx, kTileK, kTileM) ||
+        !encode_bf16_2d(&d.tm_xn[b], d.x[b], g.m, g.n, g.ldx, 64, kTileK))
+      return false;
+  }
+  d.a = reinterpret_cast<__nv_bfloat16*>(ws + g.a_off);
+  d.b = reinterpret_cast<__nv_bfloat16*>(ws + g.b_off);
+  if (!encode_bf16_2d(&d.tm_a, d.a, g.m, g.m, g.lda, kTileK, kTileM) ||
+      !encode_bf16_2d(&d.tm_b, d.b, g.m, g.m, g.lda, kTileK, kTileM))
+    return false;
+  d.rows = g.rows;
+  d.cols = g.cols;
+  d.m = g.m;
+  d.n = g.n;
+  d.ldx = g.ldx;
+  d.lda = g.lda;
+  d.transposed = g.transposed;
+  d.part_first = g.part_first;
+  d.part_count = g.part_count;
+  return true;
+}
+
+// Caller-pointer part of a matrix record; returns true if it changed.
+bool fill_caller_fields(MatDev& d, const muon_matrix_t& mt) {
+  if (d.w == mt.w && d.mom == mt.momentum && d.g == mt.grad_bf16 &&
+      d.out == mt.update_out &&
+      std::memcmp(&d.update_scale, &mt.update_scale, sizeof(float)) == 0)
+    return false;
+  d.w = mt.w;
+  d.mom = mt.momentum;
+  d.g = mt.grad_bf16;
+  d.out = mt.update_out;
+  d.update_scale = mt.update_scale;
+  return true;
+}
+
+// prologue -> K x (gram -> poly -> apply), or prologue -> final for K = 0.
+void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
+                  const float* ns_coeffs, int32_t ns_steps, float* partials,
+                  int fault, bool fresh, cudaStream_t st, Recorder* rec) {
+  HyperDev hd{h.momentum, h.lr, h.weight_decay, h.eps_row, h.eps_frob,
+              h.nesterov, h.eq_r};
+  muon_prologue_kernel<<<static_cast<unsigned>(t.n_items), kProThreads,
+                         t.pro_smem, st>>>(t.mats, t.items, hd, partials);
+  if (rec) rec->after(MUON_KIND_PROLOGUE);
+
+  if (ns_steps == 0) {
+    muon_final_noiter_kernel<<<static_cast<unsigned>(t.n_items), kProThreads, 0,
+                               st>>>(t.mats, t.items, partials, h.lr,
+                                     h.weight_decay, h.eps_frob);
+    if (rec) rec->after(MUON_KIND_FINAL);
+  }
+  for (int k = 0; k < ns_steps; ++k) {
+    NsParams p{};
+    p.mats = t.mats;
+    p.partials = partials;
+    p.err = t.err;
+    p.src = k & 1;
+    p.fault = fault;
+    p.fresh = fresh ? 1 : 0;
+    p.a = ns_coeffs[3 * k + 0];
+    p.b = ns_coeffs[3 * k + 1];
+    p.c = ns_coeffs[3 * k + 2];
+    p.lr = h.lr;
+    p.wd = h.weight_decay;
+    p.eps_frob = h.eps_frob;
+
+    p.tiles = t.gram;
+    p.n_tiles = t.n_gram;
+    p.mode = kModeGram;
+    p.first = k == 0;
+    p.last = 0;
+    ns_gemm_kernel<kGramN, false, kGramStages>
+        <<<std::min(p.n_tiles, t.num_sms), kNsThreads, GramCfg::kSmemBytes, st>>>(p);
+    if (rec) rec->after(MUON_KIND_GRAM);
+
+    p.tiles = t.poly;
+    p.n_tiles = t.n_poly;
+    p.mode = kModePoly;
+    p.first = 0;
+    p.fault = 0;
+    ns_gemm_kernel<kGramN, false, kGramStages>
+        <<<std::min(p.n_tiles, t.num_sms), kNsThreads, GramCfg::kSmemBytes, st>>>(p);
+    if (rec) rec->after(MUON_KIND_POLY);
+
+    p.tiles = t.apply;
+    p.n_tiles = t.n_apply;
+    p.mode = kModeApply;
+    p.first = k == 0;
+    p.last = k == ns_steps - 1;
+    ns_gemm_kernel<kApplyN, true, kApplyStages>
+        <<<std::min(p.n_tiles, t.num_sms), kNsThreads, ApplyCfg::kSmemBytes, st>>>(p);
+    if (rec) rec->after(MUON_KIND_APPLY);
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -428,85 +571,33 @@ muon_status_t muon_step_batched(muon_plan_t* plan, const muon_matrix_t* mats,
                                 void* workspace, size_t workspace_bytes,
                                 muon_stream_t stream) {
   // ---- validation (host, before anything is enqueued)
-  if (!plan || !mats || !hyper) return MUON_ERR_INVALID_ARG;
-  if (ns_steps < 0 || ns_steps > plan->max_ns) return MUON_ERR_UNSUPPORTED;
-  if (ns_steps > 0 && !ns_coeffs) return MUON_ERR_INVALID_ARG;
-  for (int k = 0; k < 3 * ns_steps; ++k)
-    if (!finite(ns_coeffs[k])) return MUON_ERR_INVALID_ARG;
-  const muon_hyper_t h = *hyper;
-  if (!finite(h.momentum) || !finite(h.lr) || !finite(h.weight_decay) ||
-      !finite(h.eps_row) || !finite(h.eps_frob) || h.eps_row < 0.f ||
-      h.eps_frob < 0.f || (h.nesterov != 0 && h.nesterov != 1) ||
-      (h.eq_r != 0 && h.eq_r != 1))
-    return MUON_ERR_INVALID_ARG;
+  if (!plan || !mats) return MUON_ERR_INVALID_ARG;
+  muon_status_t vs = validate_hyper(hyper, ns_coeffs, ns_steps, plan->max_ns);
+  if (vs != MUON_OK) return vs;
   if (!workspace || workspace_bytes < plan->ws_bytes) return MUON_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MUON_ERR_WORKSPACE;
   for (int i = 0; i < plan->n_mats; ++i) {
-    const muon_matrix_t& mt = mats[i];
-    const Geom& g = plan->geom[i];
-    if (mt.rows != g.rows || mt.cols != g.cols) return MUON_ERR_UNSUPPORTED;
-    if (!mt.w || !mt.momentum || !mt.grad_bf16) return MUON_ERR_INVALID_ARG;
-    if (!finite(mt.update_scale)) return MUON_ERR_INVALID_ARG;
-    if (!aligned16(mt.w) || !aligned16(mt.momentum) || !aligned16(mt.grad_bf16) ||
-        (mt.update_out && !aligned16(mt.update_out)))
-      return MUON_ERR_ALIGNMENT;
+    vs = validate_matrix(mats[i], plan->geom[i]);
+    if (vs != MUON_OK) return vs;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   // ---- per-matrix device table (uploaded only when something changed)
   char* ws = static_cast<char*>(workspace);
-  const bool reencode = plan->enc_ws != workspace;
   std::vector<MatDev>& hm = plan->h_mats;
-  if (reencode) {
-    for (int i = 0; i < plan->n_mats; ++i) {
-      const Geom& g = plan->geom[i];
-      MatDev& d = hm[i];
-      std::memset(&d, 0, sizeof(MatDev));
-      for (int b = 0; b < 2; ++b) {
-        d.x[b] = reinterpret_cast<__nv_bfloat16*>(ws + g.x_off[b]);
-        if (!encode_bf16_2d(&d.tm_xk[b], d.x[b], g.m, g.n, g.ldx, kTileK, kTileM) ||
-            !encode_bf16_2d(&d.tm_xn[b], d.x[b], g.m, g.n, g.ldx, 64, kTileK)) {
-          plan->enc_ws = nullptr;
-          plan->h_valid = false;
-          return MUON_ERR_CUDA;
-        }
-      }
-      d.a = reinterpret_cast<__nv_bfloat16*>(ws + g.a_off);
-      d.b = reinterpret_cast<__nv_bfloat16*>(ws + g.b_off);
-      if (!encode_bf16_2d(&d.tm_a, d.a, g.m, g.m, g.lda, kTileK, kTileM) ||
-          !encode_bf16_2d(&d.tm_b, d.b, g.m, g.m, g.lda, kTileK, kTileM)) {
+  if (plan->enc_ws != workspace) {
+    for (int i = 0; i < plan->n_mats; ++i)
+      if (!fill_workspace_fields(hm[i], plan->geom[i], ws)) {
         plan->enc_ws = nullptr;
         plan->h_valid = false;
         return MUON_ERR_CUDA;
       }
-      d.rows = g.rows;
-      d.cols = g.cols;
-      d.m = g.m;
-      d.n = g.n;
-      d.ldx = g.ldx;
-      d.lda = g.lda;
-      d.transposed = g.transposed;
-      d.part_first = g.part_first;
-      d.part_count = g.part_count;
-    }
     plan->enc_ws = workspace;
     plan->h_valid = false;
   }
   bool changed = !plan->h_valid;
-  for (int i = 0; i < plan->n_mats; ++i) {
-    MatDev& d = hm[i];
-    const muon_matrix_t& mt = mats[i];
-    if (d.w != mt.w || d.mom != mt.momentum ||
-        d.g != mt.grad_bf16 || d.out != mt.update_out ||
-        std::memcmp(&d.update_scale, &mt.update_scale, sizeof(float)) != 0) {
-      d.w = mt.w;
-      d.mom = mt.momentum;
-      d.g = mt.grad_bf16;
-      d.out = mt.update_out;
-      d.update_scale = mt.update_scale;
-      changed = true;
-    }
-  }
+  for (int i = 0; i < plan->n_mats; ++i)
+    changed |= fill_caller_fields(hm[i], mats[i]);
   if (changed) {
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return MUON_ERR_CUDA;
@@ -525,64 +616,15 @@ muon_status_t muon_step_batched(muon_plan_t* plan, const muon_matrix_t* mats,
   }
 
   // ---- launches
-  HyperDev hd{h.momentum, h.lr, h.weight_decay, h.eps_row, h.eps_frob,
-              h.nesterov, h.eq_r};
+  LaunchTables t{plan->d_mats, plan->d_items, static_cast<int>(plan->items.size()),
+                 plan->d_gram, static_cast<int>(plan->gram.size()),
+                 plan->d_poly, static_cast<int>(plan->poly.size()),
+                 plan->d_apply, static_cast<int>(plan->apply.size()),
+                 plan->d_err, plan->num_sms, plan->pro_smem};
   float* partials = reinterpret_cast<float*>(ws + plan->part_off);
   Recorder rec(plan, st);
-
-  muon_prologue_kernel<<<static_cast<unsigned>(plan->items.size()), kProThreads,
-                         plan->pro_smem, st>>>(plan->d_mats, plan->d_items, hd,
-                                               partials);
-  rec.after(MUON_KIND_PROLOGUE);
-
-  if (ns_steps == 0) {
-    muon_final_noiter_kernel<<<static_cast<unsigned>(plan->items.size()),
-                               kProThreads, 0, st>>>(
-        plan->d_mats, plan->d_items, partials, h.lr, h.weight_decay, h.eps_frob);
-    rec.after(MUON_KIND_FINAL);
-  }
-  for (int k = 0; k < ns_steps; ++k) {
-    NsParams p{};
-    p.mats = plan->d_mats;
-    p.partials = partials;
-    p.err = plan->d_err;
-    p.src = k & 1;
-    p.fault = plan->fault;
-    p.fresh = changed ? 1 : 0;
-    p.a = ns_coeffs[3 * k + 0];
-    p.b = ns_coeffs[3 * k + 1];
-    p.c = ns_coeffs[3 * k + 2];
-    p.lr = h.lr;
-    p.wd = h.weight_decay;
-    p.eps_frob = h.eps_frob;
-
-    p.tiles = plan->d_gram;
-    p.n_tiles = static_cast<int>(plan->gram.size());
-    p.mode = kModeGram;
-    p.first = k == 0;
-    p.last = 0;
-    ns_gemm_kernel<kGramN, false, kGramStages>
-        <<<std::min(p.n_tiles, plan->num_sms), 192, GramCfg::kSmemBytes, st>>>(p);
-    rec.after(MUON_KIND_GRAM);
-
-    p.tiles = plan->d_poly;
-    p.n_tiles = static_cast<int>(plan->poly.size());
-    p.mode = kModePoly;
-    p.first = 0;
-    p.fault = 0;
-    ns_gemm_kernel<kGramN, false, kGramStages>
-        <<<std::min(p.n_tiles, plan->num_sms), 192, GramCfg::kSmemBytes, st>>>(p);
-    rec.after(MUON_KIND_POLY);
-
-    p.tiles = plan->d_apply;
-    p.n_tiles = static_cast<int>(plan->apply.size());
-    p.mode = kModeApply;
-    p.first = k == 0;
-    p.last = k == ns_steps - 1;
-    ns_gemm_kernel<kApplyN, true, kApplyStages>
-        <<<std::min(p.n_tiles, plan->num_sms), 192, ApplyCfg::kSmemBytes, st>>>(p);
-    rec.after(MUON_KIND_APPLY);
-  }
+  enqueue_step(t, *hyper, ns_coeffs, ns_steps, partials, plan->fault, changed, st,
+               plan->timing ? &rec : nullptr);
   rec.finish();
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;

@@ -64,7 +64,8 @@ def test_constants(L):
     assert binding.status_string(-99) == "unknown status"
     assert L.muon_step_launches(5) == 16
     assert L.muon_step_launches(0) == 2
-    assert L.ema_update_launches(278) == 3
+    assert L.ema_update_launches(278) == 1
+    assert L.ema_update_launches(321) == 2
     assert L.ema_update_launches(0) == 0
     assert L.muon_plan_workspace_bytes(None) == 0
 
