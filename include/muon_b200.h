@@ -172,6 +172,43 @@ muon_status_t muon_plan_set_fault(muon_plan_t *plan, int32_t fault);
 /* ABI version (major * 100 + minor). */
 int32_t muon_abi_version(void);
 
+/* ---- One batched step without any device allocation ----------------------
+ * The pages have no counterpart to this call.  It is for callers that cannot
+ * allocate device memory: a framework that owns every device allocation
+ * through its own pool and hands a plug-in only its inputs and outputs, or a
+ * latency-critical loop that forbids cudaMalloc after start-up (cudaMalloc
+ * can synchronise the device and stall other streams).  Such a caller can
+ * neither create a plan (muon_plan_create allocates the plan's table) nor
+ * provide a workspace.
+ *
+ * It computes the same step as muon_step_batched on the same kernels.  Its
+ * scratch -- the per-matrix table with the TMA descriptors, the work and tile
+ * lists, the error word, X, A, B' and the norm partials -- lives in one
+ * file-scope device array of MUON_NOALLOC_SCRATCH_BYTES, which every device
+ * that loads this library's kernels holds until the process exits.
+ *  mats: host array of n_mats matrices (1 <= n_mats <= MUON_NOALLOC_MAX_MATS),
+ *        same rules as muon_step_batched; ns_steps in [0, 16].
+ *  Returns MUON_ERR_WORKSPACE if the batch needs more scratch than the array
+ *  holds (the array fits, e.g., one 11L x 512d layer or any single matrix
+ *  up to 1024 x 4096), MUON_ERR_UNSUPPORTED beyond the count limits.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and sets kernel attributes; make that first call
+ * before any stream capture.  Every call re-uploads its tables with
+ * cudaMemcpyAsync from pageable host memory (so it cannot be captured), clears
+ * the error word with cudaMemsetAsync, and calls no cudaMalloc, cudaFree or
+ * other allocating routine.  All calls share the one array: calls that overlap
+ * on the GPU (different streams, or different host threads without ordering)
+ * race on it; order them on one stream.  Device-side wait timeouts in this
+ * path set the array's error word but are not reported back to the host. */
+#define MUON_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+#define MUON_NOALLOC_MAX_MATS 64
+muon_status_t muon_step_batched_noalloc(const muon_matrix_t *mats,
+                                        int32_t n_mats,
+                                        const muon_hyper_t *hyper,
+                                        const float *ns_coeffs,
+                                        int32_t ns_steps,
+                                        muon_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -92,6 +92,11 @@ def lib():
     L.muon_plan_set_fault.restype = c_int32
     L.muon_abi_version.argtypes = []
     L.muon_abi_version.restype = c_int32
+    L.muon_step_batched_noalloc.argtypes = [POINTER(muon_matrix_t), c_int32,
+                                            POINTER(muon_hyper_t),
+                                            POINTER(c_float), c_int32,
+                                            c_void_p]
+    L.muon_step_batched_noalloc.restype = c_int32
     _lib = L
     return L
 
@@ -291,3 +296,45 @@ def step_launches(ns_steps: int) -> int:
 
 def ema_launches(n_tensors: int) -> int:
     return int(lib().ema_update_launches(int(n_tensors)))
+
+
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+NOALLOC_MAX_MATS = 64
+
+
+def muon_step_batched_noalloc(weights, momenta, grads, hyper, coeffs,
+                              update_scales: Optional[Sequence[float]] = None,
+                              update_out=None, stream=None):
+    """One batched Muon step through muon_step_batched_noalloc: no plan and
+    no workspace; the library's fixed device scratch array is used instead
+    (for callers that cannot allocate device memory).  Same tensor rules as
+    MuonPlan.step."""
+    import torch
+    n = len(weights)
+    if not (len(momenta) == len(grads) == n):
+        raise ValueError("one weight, momentum and gradient per matrix")
+    mats = (muon_matrix_t * max(n, 1))()
+    for i in range(n):
+        r, c = (int(v) for v in weights[i].shape)
+        _check_tensor(weights[i], torch.float32, (r, c), f"weights[{i}]")
+        _check_tensor(momenta[i], torch.float32, (r, c), f"momenta[{i}]")
+        _check_tensor(grads[i], torch.bfloat16, (r, c), f"grads[{i}]")
+        o = update_out[i] if update_out is not None else None
+        if o is not None:
+            _check_tensor(o, torch.float32, (r, c), f"update_out[{i}]")
+        s = (update_scales[i] if update_scales is not None
+             else max(1.0, r / c) ** 0.5)
+        mats[i] = muon_matrix_t(weights[i].data_ptr(), momenta[i].data_ptr(),
+                                grads[i].data_ptr(),
+                                o.data_ptr() if o is not None else None,
+                                r, c, float(s))
+    hp = muon_hyper_t(float(hyper.momentum), float(hyper.lr),
+                      float(hyper.weight_decay), float(hyper.eps_row),
+                      float(hyper.eps_frob), int(bool(hyper.nesterov)),
+                      int(bool(hyper.eq_r)))
+    flat = [float(v) for row in coeffs for v in row]
+    carr = (c_float * max(len(flat), 1))(*flat)
+    _check(lib().muon_step_batched_noalloc(mats, n, ctypes.byref(hp), carr,
+                                           len(flat) // 3,
+                                           _stream_handle(stream)),
+           "muon_step_batched_noalloc")

@@ -13,6 +13,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -673,6 +674,231 @@ muon_status_t ema_update_batched(float* const* ema, const float* const* params,
     const unsigned grid = static_cast<unsigned>(std::min<long long>(want, 8ll * sms));
     ema_update_kernel<<<grid, kEmaThreads, 0, st>>>(p);
   }
+  if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
+  return MUON_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// muon_step_batched_noalloc: the batched step for callers that cannot
+// allocate device memory.
+//
+// All of the step's scratch (the per-matrix records with their TMA
+// descriptors, the work and tile lists, the error word, and the working
+// matrices X, A, B' and the norm partials) lives in one file-scope device
+// array, g_noalloc_scratch, of MUON_NOALLOC_SCRATCH_BYTES.  The CUDA runtime
+// reserves it on every device where this library's kernels are loaded, for
+// the life of the process.  Host code must not pass the array's name to a
+// kernel (in host code it names a host-side stand-in); the device address
+// comes from cudaGetSymbolAddress, looked up once per device with that
+// device current, on the first call made on that device.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char
+    g_noalloc_scratch[MUON_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kNoAllocMaxDevices = 64;
+constexpr int kNoAllocMaxItems = 8192;
+constexpr int kNoAllocMaxGramTiles = 4096;
+constexpr int kNoAllocMaxApplyTiles = 8192;
+
+// Device address of g_noalloc_scratch per device (filled on first use).
+void* g_noalloc_dev_ptr[kNoAllocMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+// Host-side staging of the tables (fixed capacity; guarded by the mutex).
+Geom g_na_geom[MUON_NOALLOC_MAX_MATS];
+MatDev g_na_mats[MUON_NOALLOC_MAX_MATS];
+ProItem g_na_items[kNoAllocMaxItems];
+NsTile g_na_gram[kNoAllocMaxGramTiles];
+NsTile g_na_poly[kNoAllocMaxGramTiles];
+NsTile g_na_apply[kNoAllocMaxApplyTiles];
+
+NsTile g_na_tmp[kNoAllocMaxApplyTiles];
+
+// Tile order: longest K first, list order among equal K (the order the
+// plan's stable sort gives), without a heap buffer: one pass per distinct K
+// length, from the longest down.
+void sort_tiles_by_k(NsTile* v, int n) {
+  int out = 0;
+  int cur = 1 << 30;
+  while (out < n) {
+    int next = -1;
+    for (int i = 0; i < n; ++i)
+      if (v[i].kt < cur && v[i].kt > next) next = v[i].kt;
+    for (int i = 0; i < n; ++i)
+      if (v[i].kt == next) g_na_tmp[out++] = v[i];
+    cur = next;
+  }
+  std::memcpy(v, g_na_tmp, sizeof(NsTile) * n);
+}
+
+}  // namespace
+
+extern "C" {
+
+muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
+                                        int32_t n_mats,
+                                        const muon_hyper_t* hyper,
+                                        const float* ns_coeffs,
+                                        int32_t ns_steps,
+                                        muon_stream_t stream) {
+  if (!mats || n_mats < 1) return MUON_ERR_INVALID_ARG;
+  if (n_mats > MUON_NOALLOC_MAX_MATS) return MUON_ERR_UNSUPPORTED;
+  muon_status_t vs = validate_hyper(hyper, ns_coeffs, ns_steps, kMaxNsSteps);
+  if (vs != MUON_OK) return vs;
+
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+
+  // Geometry and lists into the fixed host tables.
+  size_t off = 0;
+  int n_items = 0, n_gram = 0, n_apply = 0;
+  size_t pro_smem = 0;
+  for (int i = 0; i < n_mats; ++i) {
+    const int rows = mats[i].rows, cols = mats[i].cols;
+    if (rows < 1 || cols < 1) return MUON_ERR_INVALID_ARG;
+    if (rows > (1 << 20) || cols > (1 << 20) ||
+        static_cast<long long>(rows) * cols > (1ll << 31) - 1)
+      return MUON_ERR_UNSUPPORTED;
+    Geom& g = g_na_geom[i];
+    g.rows = rows;
+    g.cols = cols;
+    g.transposed = rows > cols;
+    g.m = std::min(rows, cols);
+    g.n = std::max(rows, cols);
+    g.ldx = static_cast<int>(align_up(g.n, 8));
+    g.lda = static_cast<int>(align_up(g.m, 8));
+    for (int b = 0; b < 2; ++b) {
+      g.x_off[b] = off;
+      off = align_up(off + static_cast<size_t>(g.m) * g.ldx * 2, 1024);
+    }
+    g.a_off = off;
+    off = align_up(off + static_cast<size_t>(g.m) * g.lda * 2, 1024);
+    g.b_off = off;
+    off = align_up(off + static_cast<size_t>(g.m) * g.lda * 2, 1024);
+    vs = validate_matrix(mats[i], g);
+    if (vs != MUON_OK) return vs;
+
+    const int rt = pro_rows_per_item(g.rows, g.cols);
+    g.part_first = n_items;
+    for (int r0 = 0; r0 < g.rows; r0 += rt) {
+      if (n_items >= kNoAllocMaxItems) return MUON_ERR_UNSUPPORTED;
+      g_na_items[n_items++] = ProItem{i, r0, std::min(rt, g.rows - r0), 0};
+    }
+    g.part_count = n_items - g.part_first;
+    if (g.transposed)
+      pro_smem = std::max(pro_smem, static_cast<size_t>(rt) * (g.cols + 2) * 2);
+
+    const int tm = ceil_div(g.m, kTileM);
+    for (int ti = 0; ti < tm; ++ti)
+      for (int tj = ti; tj < tm; ++tj) {
+        if (n_gram >= kNoAllocMaxGramTiles) return MUON_ERR_UNSUPPORTED;
+        g_na_gram[n_gram] = NsTile{static_cast<uint16_t>(i), static_cast<uint16_t>(ti),
+                                   static_cast<uint16_t>(tj),
+                                   static_cast<uint16_t>(ceil_div(g.n, kTileK))};
+        g_na_poly[n_gram] = NsTile{static_cast<uint16_t>(i), static_cast<uint16_t>(ti),
+                                   static_cast<uint16_t>(tj),
+                                   static_cast<uint16_t>(ceil_div(g.m, kTileK))};
+        ++n_gram;
+      }
+    const int tn = ceil_div(g.n, kApplyN);
+    for (int ti = 0; ti < tm; ++ti)
+      for (int tj = 0; tj < tn; ++tj) {
+        if (n_apply >= kNoAllocMaxApplyTiles) return MUON_ERR_UNSUPPORTED;
+        g_na_apply[n_apply++] = NsTile{static_cast<uint16_t>(i), static_cast<uint16_t>(ti),
+                                       static_cast<uint16_t>(tj),
+                                       static_cast<uint16_t>(ceil_div(g.m, kTileK))};
+      }
+  }
+  sort_tiles_by_k(g_na_gram, n_gram);
+  sort_tiles_by_k(g_na_poly, n_gram);
+  sort_tiles_by_k(g_na_apply, n_apply);
+  const size_t part_off = off;
+  off = align_up(off + static_cast<size_t>(n_items) * sizeof(float), 1024);
+  const size_t ws_bytes = off;
+
+  // Layout of the device array: [error word][tables][workspace].
+  size_t t_off = 256;
+  const size_t mats_off = t_off;
+  t_off = align_up(t_off + sizeof(MatDev) * n_mats, 256);
+  const size_t items_off = t_off;
+  t_off = align_up(t_off + sizeof(ProItem) * n_items, 256);
+  const size_t gram_off = t_off;
+  t_off = align_up(t_off + sizeof(NsTile) * n_gram, 256);
+  const size_t poly_off = t_off;
+  t_off = align_up(t_off + sizeof(NsTile) * n_gram, 256);
+  const size_t apply_off = t_off;
+  t_off = align_up(t_off + sizeof(NsTile) * n_apply, 1024);
+  const size_t ws_off = t_off;
+  if (ws_off + ws_bytes > MUON_NOALLOC_SCRATCH_BYTES) return MUON_ERR_WORKSPACE;
+
+  // Device address of the array on the current device (once per device).
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MUON_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return MUON_ERR_UNSUPPORTED;
+  if (!g_noalloc_dev_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+      cudaGetLastError();
+      return MUON_ERR_CUDA;
+    }
+    if (cudaFuncSetAttribute(ns_gemm_kernel<kGramN, false, kGramStages>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(GramCfg::kSmemBytes)) != cudaSuccess ||
+        cudaFuncSetAttribute(ns_gemm_kernel<kApplyN, true, kApplyStages>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(ApplyCfg::kSmemBytes)) != cudaSuccess) {
+      cudaGetLastError();
+      return MUON_ERR_CUDA;
+    }
+    g_noalloc_dev_ptr[dev] = ptr;
+  }
+  int num_sms = 148;
+  if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) !=
+      cudaSuccess)
+    return MUON_ERR_CUDA;
+  if (pro_smem > 48 * 1024 &&
+      cudaFuncSetAttribute(muon_prologue_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(pro_smem)) != cudaSuccess) {
+    cudaGetLastError();
+    return MUON_ERR_CUDA;
+  }
+  char* base = static_cast<char*>(g_noalloc_dev_ptr[dev]);
+  char* ws = base + ws_off;
+  for (int i = 0; i < n_mats; ++i) {
+    if (!fill_workspace_fields(g_na_mats[i], g_na_geom[i], ws)) return MUON_ERR_CUDA;
+    fill_caller_fields(g_na_mats[i], mats[i]);
+  }
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The array keeps the previous call's contents: the error word must start
+  // at zero; everything else is written before it is read.
+  if (cudaMemsetAsync(base, 0, sizeof(int32_t), st) != cudaSuccess ||
+      cudaMemcpyAsync(base + mats_off, g_na_mats, sizeof(MatDev) * n_mats,
+                      cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(base + items_off, g_na_items, sizeof(ProItem) * n_items,
+                      cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(base + gram_off, g_na_gram, sizeof(NsTile) * n_gram,
+                      cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(base + poly_off, g_na_poly, sizeof(NsTile) * n_gram,
+                      cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(base + apply_off, g_na_apply, sizeof(NsTile) * n_apply,
+                      cudaMemcpyHostToDevice, st) != cudaSuccess) {
+    cudaGetLastError();
+    return MUON_ERR_CUDA;
+  }
+
+  LaunchTables t{reinterpret_cast<const MatDev*>(base + mats_off),
+                 reinterpret_cast<const ProItem*>(base + items_off), n_items,
+                 reinterpret_cast<const NsTile*>(base + gram_off), n_gram,
+                 reinterpret_cast<const NsTile*>(base + poly_off), n_gram,
+                 reinterpret_cast<const NsTile*>(base + apply_off), n_apply,
+                 reinterpret_cast<int32_t*>(base), num_sms, pro_smem};
+  float* partials = reinterpret_cast<float*>(ws + part_off);
+  enqueue_step(t, *hyper, ns_coeffs, ns_steps, partials, 0, true, st, nullptr);
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
 }
