@@ -154,13 +154,16 @@ typedef enum {
   MUON_KIND_POLY = 2,     /* B = b A + c A A                               */
   MUON_KIND_APPLY = 3,    /* X <- a X + B X (and, last step, W update)     */
   MUON_KIND_FINAL = 4,    /* ns_steps == 0: W update from the normalised X */
-  MUON_KIND_COUNT = 5
+  MUON_KIND_NS = 5,       /* all ns_steps Newton-Schulz steps, one launch:
+                             gram, poly and apply tiles of every matrix and
+                             step, and the weight update of the last step  */
+  MUON_KIND_COUNT = 6
 } muon_kind_t;
 muon_status_t muon_plan_set_timing(muon_plan_t *plan, int32_t enable);
 muon_status_t muon_plan_timing_read(muon_plan_t *plan, int32_t *launches,
                                     double *ms, int32_t n_kinds);
 
-/* Launch counts of one call with ns_steps steps (for launch accounting). */
+/* Kernel launches of one call with ns_steps steps (for launch accounting). */
 int32_t muon_step_launches(int32_t ns_steps);
 int32_t ema_update_launches(int32_t n_tensors);
 

@@ -1,0 +1,500 @@
+// All K Newton-Schulz steps of every matrix in one persistent launch on CTA
+// pairs (tcgen05.mma.cta_group::2, 256 x 256 tiles).
+//
+// The work list is, for k = 0..K-1: the gram tiles of every matrix, then the
+// poly tiles, then the apply tiles.  Cluster c takes items c, c + C, c + 2C,
+// ... in that order.  An item waits (in its producer, before loading) until
+// the phase it reads is complete for its matrix:
+//   gram(k)  reads X_k   <- every apply(k-1) tile of the matrix (k > 0)
+//   poly(k)  reads A     <- every gram(k) tile of the matrix
+//   apply(k) reads B', X <- every poly(k) tile of the matrix
+// Completion is counted per (matrix, step, phase) in global memory: each CTA
+// adds 1 after its half of a tile is stored (release), producers spin with
+// acquire loads (bounded).  Every dependency precedes its dependants in the
+// list and every cluster walks the list in order, so with all clusters
+// resident the schedule cannot deadlock.  Different matrices overlap freely,
+// and a tile's epilogue overlaps the next item's loads and MMAs.
+//
+// Per item:
+//   gram  A  = s^2 X X^T   (upper pair tiles; off-diagonal ones also stored
+//                          mirrored, so A is complete for its consumers)
+//   poly  B' = a I + b A + c A A   (A symmetric, so A A = A A^T)
+//   apply X <- s B' X      (last step: W <- W (1 - lr wd) - lr scale O)
+// X <- a X + B X is evaluated as (a I + B) X: one product, and the bf16 copy
+// of B' holds a + B on its diagonal instead of the cancelling pair.
+// s = 1 / (||X~||_F + eps_frob) in step 0 (the Frobenius normalisation folded
+// into the first products), 1 afterwards.
+//
+// Roles (320 threads per CTA): warp 0 issues TMA loads (.cta_group::2, no
+// multicast) into a 6-stage ring, counting both CTAs' bytes on the leader's
+// barrier; warp 1 of the leader issues the pair MMAs from one thread and
+// frees stages / hands over accumulators with multicast tcgen05.commit;
+// warps 2-9 of each CTA drain that CTA's 128 TMEM lanes and run the fused
+// epilogue.  All waits are bounded: a failure raises both CTAs' abort flags
+// and the global error word, and every CTA still meets the final cluster
+// barrier before TMEM is freed.
+//
+// Source of the step: PR #1396 "Record: Combined 3-Layer Recurrence +
+// Parallel Residuals + Polar Express + Brotli", table "Techniques Combined",
+// row "Polar Express Newton-Schulz"; PR #1584 "Record: Improved Parallel
+// Residuals + Systems Optimization", section "Summary" (fused Muon kernel).
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "k_ns_common.cuh"
+#include "k_ns_gemm_pair.cuh"
+#include "muon_types.cuh"
+#include "sm100_ptx.cuh"
+
+namespace muonb200 {
+
+constexpr int kMegaMaxSteps = 16;
+constexpr int kMegaStages = 6;
+
+struct MegaParams {
+  const MatDev* mats;
+  const NsTile* gram;     // pair tiles, K = n
+  const NsTile* poly;     // pair tiles, K = m
+  const NsTile* apply;    // pair tiles, K = m
+  const float* partials;
+  int32_t* err;
+  int32_t* done;          // [mat][step][phase] completion counts, zeroed
+  int32_t n_gram, n_poly, n_apply;
+  int32_t steps;
+  int32_t fault, fresh;
+  float a[kMegaMaxSteps], b[kMegaMaxSteps], c[kMegaMaxSteps];
+  float lr, wd, eps_frob;
+};
+
+using MegaCfg = PairCfg<false, kMegaStages>;   // 32 KB stages + transpose buffers
+// two more barriers than PairCfg (the epilogue completion pair), plus slack
+constexpr size_t kMegaSmemBytes = MegaCfg::kSmemBytes + 64;
+
+// Spins (acquire) until *ctr >= target.  Gives up on the CTA's abort flag,
+// on a non-zero global error word (another CTA failed) or after the limit.
+__device__ __forceinline__ bool wait_count(const int32_t* ctr, int32_t target,
+                                           volatile int* abort_flag,
+                                           const int32_t* err) {
+  if (ld_acquire_gpu(ctr) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    if ((i & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (*reinterpret_cast<const volatile int32_t*>(err) != 0) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    __nanosleep(64);
+  }
+}
+
+struct MegaItem {
+  NsTile tl;
+  int mode;
+  int k;
+};
+
+__device__ __forceinline__ MegaItem mega_item(const MegaParams& p, int g) {
+  const int per_step = p.n_gram + p.n_poly + p.n_apply;
+  MegaItem it;
+  it.k = g / per_step;
+  int r = g - it.k * per_step;
+  if (r < p.n_gram) {
+    it.mode = kModeGram;
+    it.tl = p.gram[r];
+  } else if (r < p.n_gram + p.n_poly) {
+    it.mode = kModePoly;
+    it.tl = p.poly[r - p.n_gram];
+  } else {
+    it.mode = kModeApply;
+    it.tl = p.apply[r - p.n_gram - p.n_poly];
+  }
+  return it;
+}
+
+__device__ __forceinline__ int32_t* done_counter(const MegaParams& p, int mat,
+                                                 int k, int mode) {
+  return p.done + (static_cast<size_t>(mat) * p.steps + k) * 3 + mode;
+}
+
+// Completion count an item must see before it reads its inputs; nullptr if
+// it has no in-kernel dependency (gram of step 0 reads the prologue's X).
+__device__ __forceinline__ const int32_t* dep_counter(const MegaParams& p,
+                                                      const MegaItem& it,
+                                                      const MatDev* md,
+                                                      int32_t& target) {
+  if (it.mode == kModeGram) {
+    if (it.k == 0) return nullptr;
+    target = 2 * md->n_apply_tiles;
+    return done_counter(p, it.tl.mat, it.k - 1, kModeApply);
+  }
+  target = 2 * md->n_sym_tiles;
+  return done_counter(p, it.tl.mat, it.k, it.mode == kModePoly ? kModeGram : kModePoly);
+}
+
+__global__ void __launch_bounds__(kNsThreads, 1)
+ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
+  using Cfg = MegaCfg;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __nv_bfloat16* xpose =
+      reinterpret_cast<__nv_bfloat16*>(smem + kMegaStages * Cfg::kStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      smem + kMegaStages * Cfg::kStageBytes + Cfg::kXposeBytes);
+  // bars: full[S], empty[S], tfull[2], tempty[2], drain, epi[2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::kNumBars + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  constexpr int S = kMegaStages;
+
+  const uint32_t smem0 = smem_addr(smem);
+  auto sA = [&](int s) { return smem0 + s * Cfg::kStageBytes; };
+  auto sB = [&](int s) { return smem0 + s * Cfg::kStageBytes + Cfg::kABytes; };
+  auto full_bar = [&](int s) { return smem_addr(bars + s); };
+  auto empty_bar = [&](int s) { return smem_addr(bars + S + s); };
+  auto tfull_bar = [&](int a) { return smem_addr(bars + 2 * S + a); };
+  auto tempty_bar = [&](int a) { return smem_addr(bars + 2 * S + 2 + a); };
+  const uint32_t drain_bar = smem_addr(bars + 2 * S + 4);
+  auto epi_bar = [&](int a) { return smem_addr(bars + 2 * S + 5 + a); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  const int total = p.steps * (p.n_gram + p.n_poly + p.n_apply);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 2 * kEpiWarps);
+      mbar_init(epi_bar(a), kEpiWarps);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_addr(tmem_slot), Cfg::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t peer_abort = mapa_shared(smem_addr(const_cast<int*>(abort_flag)), rank ^ 1u);
+  const uint32_t leader_full0 = mapa_shared(full_bar(0), 0);
+  auto fail = [&](int32_t code) {
+    atomicCAS(p.err, 0, code);
+    *abort_flag = 1;
+    st_shared_cluster_u32(peer_abort, 1u);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int g = pair; ok && g < total; g += npairs) {
+        const MegaItem item = mega_item(p, g);
+        const NsTile tl = item.tl;
+        const MatDev* md = p.mats + tl.mat;
+        const int src = item.k & 1;
+        const CUtensorMap* tm_a;
+        const CUtensorMap* tm_b;
+        if (item.mode == kModeGram) {
+          tm_a = &md->tm_xk[src];
+          tm_b = tm_a;
+        } else if (item.mode == kModePoly) {
+          tm_a = &md->tm_a;
+          tm_b = tm_a;
+        } else {
+          tm_a = &md->tm_b;
+          tm_b = &md->tm_xn[src];
+        }
+        if (p.fresh) {
+          tensormap_acquire(tm_a);
+          if (tm_b != tm_a) tensormap_acquire(tm_b);
+        }
+        int32_t target = 0;
+        const int32_t* dep = dep_counter(p, item, md, target);
+        if (dep != nullptr) {
+          if (!wait_count(dep, target, abort_flag, p.err)) {
+            fail(kErrTimeoutProducer);
+            ok = false;
+            break;
+          }
+          fence_proxy_async_global();   // generic stores of other CTAs -> TMA reads
+        }
+        const int arow = tl.ti * kPairTile + static_cast<int>(rank) * 128;
+        const int bcol = tl.tj * kPairTile + static_cast<int>(rank) * 128;
+        for (int kb = 0; kb < tl.kt; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag)) {
+            fail(kErrTimeoutProducer);
+            ok = false;
+            break;
+          }
+          if (p.fault == 1 && pair == 0 && it == 0 && leader) continue;  // test hook
+          if (leader) mbar_arrive_expect_tx(full_bar(s), Cfg::kTxBytes);
+          const uint32_t lfull = leader_full0 + 8u * s;
+          tma_load_2d_pair(sA(s), tm_a, lfull, kb * kTileK, arow);
+          if (item.mode != kModeApply) {
+            tma_load_2d_pair(sB(s), tm_b, lfull, kb * kTileK, bcol);
+          } else {
+            tma_load_2d_pair(sB(s), tm_b, lfull, bcol, kb * kTileK);
+            tma_load_2d_pair(sB(s) + 64 * kTileK * 2, tm_b, lfull, bcol + 64,
+                             kb * kTileK);
+          }
+        }
+      }
+      if (!ok) {
+        volatile int never = 0;
+        if (leader)
+          for (int j = (it > S ? it - S : 0); j < it; ++j)
+            mbar_wait_bounded(full_bar(j % S), (j / S) & 1, &never,
+                              10ull * 1000ull * 1000ull);
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 20000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc_k = idesc_bf16_f32_pair(kPairTile, false);
+      constexpr uint32_t idesc_mn = idesc_bf16_f32_pair(kPairTile, true);
+      int it = 0, lt = 0;
+      bool ok = true;
+      for (int g = pair; ok && g < total; g += npairs, ++lt) {
+        const MegaItem item = mega_item(p, g);
+        const bool bmn = item.mode == kModeApply;
+        const uint32_t idesc = bmn ? idesc_mn : idesc_k;
+        const int acc = lt & 1;
+        const uint32_t aph = (lt >> 1) & 1;
+        if (!mbar_wait_bounded(tempty_bar(acc), aph ^ 1u, abort_flag)) {
+          fail(kErrTimeoutMma);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kPairTile;
+        for (int kb = 0; kb < item.tl.kt; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (!mbar_wait_bounded(full_bar(s), ph, abort_flag)) {
+            fail(kErrTimeoutMma);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kTileK / 16; ++kk) {
+            const uint64_t adesc = smem_desc_sw128(sA(s) + kk * 32, 16, 1024);
+            const uint64_t bdesc =
+                bmn ? smem_desc_sw128(sB(s) + kk * 2048, 64 * kTileK * 2, 1024)
+                    : smem_desc_sw128(sB(s) + kk * 32, 16, 1024);
+            umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit_pair_mc(empty_bar(s), 0x3);
+        }
+        if (!ok) break;
+        umma_commit_pair_mc(tfull_bar(acc), 0x3);
+      }
+      umma_commit_pair_mc(drain_bar, 0x1);
+      volatile int never = 0;
+      mbar_wait_bounded(drain_bar, 0, &never, 10ull * 1000ull * 1000ull);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;
+    const int quad = warp & 3;
+    const int half = ew >> 2;
+    const int r_pair = static_cast<int>(rank) * 128 + quad * 32 + lane;
+    __nv_bfloat16* xbuf = xpose + ew * 32 * kXposeLd;
+    const uint32_t leader_tempty0 = mapa_shared(tempty_bar(0), 0);
+    const bool signaler = ew == 0 && lane == 0;
+    int lt = 0;
+    for (int g = pair; g < total; g += npairs, ++lt) {
+      const MegaItem item = mega_item(p, g);
+      const NsTile tl = item.tl;
+      const MatDev* md = p.mats + tl.mat;
+      const int acc = lt & 1;
+      const uint32_t aph = (lt >> 1) & 1;
+      if (!mbar_wait_bounded(tfull_bar(acc), aph, abort_flag)) {
+        fail(kErrTimeoutEpilogue);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                             static_cast<uint32_t>(acc * kPairTile);
+      const int row0 = tl.ti * kPairTile + static_cast<int>(rank) * 128 + quad * 32;
+      const int row = row0 + lane;
+      const int m = md->m;
+      const bool row_ok = row < m;
+      const bool first = item.k == 0;
+      const bool last = item.k == p.steps - 1;
+      const float s = first ? frob_scale(md, p.partials, p.eps_frob) : 1.f;
+
+      if (item.mode == kModeGram || item.mode == kModePoly) {
+        __nv_bfloat16* outp = (item.mode == kModeGram) ? md->a : md->b;
+        const bool diag_tile = tl.ti == tl.tj;
+        if (item.mode == kModePoly) {
+          // The generic reads of A below need the gram stores of other CTAs.
+          if (lane == 0) {
+            int32_t target = 2 * md->n_sym_tiles;
+            wait_count(done_counter(p, tl.mat, item.k, kModeGram), target,
+                       abort_flag, p.err);
+          }
+          __syncwarp();
+        }
+        const float pa = p.a[item.k], pb = p.b[item.k], pc = p.c[item.k];
+#pragma unroll 1
+        for (int cc = half; cc < kPairTile / 32; cc += 2) {
+          const int col0 = tl.tj * kPairTile + cc * 32;
+          float av[32];
+          if (item.mode == kModePoly && row_ok)
+            load_row32_bf16(md->a + static_cast<size_t>(row) * md->lda, col0, m, av);
+          float v[32];
+          tmem_load_32cols(tbase + cc * 32, v);
+          if (item.mode == kModeGram) {
+            const float s2 = s * s;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] *= s2;
+          } else if (row_ok) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = fmaf(pb, av[e], pc * v[e]);
+            if (diag_tile && (r_pair >> 5) == cc) {
+              const int d = r_pair & 31;
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (e == d) v[e] += pa;
+            }
+          }
+          if (row_ok)
+            store_row32_bf16(outp + static_cast<size_t>(row) * md->lda, col0, m, v);
+          if (!diag_tile)
+            store_mirror32_bf16(outp, md->lda, row0, col0, m, lane, xbuf, v);
+        }
+      } else {
+        const int n = md->n;
+        __nv_bfloat16* xd = md->x[(item.k & 1) ^ 1] + static_cast<size_t>(row) * md->ldx;
+        const float decay = 1.f - p.lr * p.wd;
+        const float step = p.lr * md->update_scale;
+        const bool tr = md->transposed != 0;
+#pragma unroll 1
+        for (int cc = half; cc < kPairTile / 32; cc += 2) {
+          const int col0 = tl.tj * kPairTile + cc * 32;
+          const bool live = row_ok && col0 < n;
+          float wv[32];
+          float* w_row = nullptr;
+          const bool wvec = !tr && col0 + 32 <= n && (n & 3) == 0;
+          if (last && live) {
+            if (!tr) {
+              w_row = md->w + static_cast<size_t>(row) * n + col0;
+              if (wvec) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                  const float4 w4 = reinterpret_cast<const float4*>(w_row)[q];
+                  wv[4 * q] = w4.x; wv[4 * q + 1] = w4.y;
+                  wv[4 * q + 2] = w4.z; wv[4 * q + 3] = w4.w;
+                }
+              } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) wv[e] = col0 + e < n ? w_row[e] : 0.f;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                wv[e] = col0 + e < n
+                            ? md->w[static_cast<size_t>(col0 + e) * m + row] : 0.f;
+            }
+          }
+          float v[32];
+          tmem_load_32cols(tbase + cc * 32, v);
+          if (!live) continue;
+          if (first) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] *= s;
+          }
+          if (!last) {
+            store_row32_bf16(xd, col0, n, v);
+            continue;
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) wv[e] = fmaf(wv[e], decay, -step * v[e]);
+          if (!tr) {
+            float* o = md->out ? md->out + static_cast<size_t>(row) * n + col0 : nullptr;
+            if (wvec) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                reinterpret_cast<float4*>(w_row)[q] =
+                    make_float4(wv[4 * q], wv[4 * q + 1], wv[4 * q + 2], wv[4 * q + 3]);
+                if (o)
+                  reinterpret_cast<float4*>(o)[q] =
+                      make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (col0 + e < n) {
+                  w_row[e] = wv[e];
+                  if (o) o[e] = v[e];
+                }
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (col0 + e < n) {
+                const size_t off = static_cast<size_t>(col0 + e) * m + row;
+                md->w[off] = wv[e];
+                if (md->out) md->out[off] = v[e];
+              }
+          }
+        }
+      }
+      // Accumulator free: the leader may start the item after next.
+      tc_fence_before();
+      // Outputs of this item visible (to TMA readers too) before counting it.
+      fence_proxy_async_global();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(tempty_bar(acc));
+        else mbar_arrive_cluster(leader_tempty0 + 8u * acc);
+        mbar_arrive(epi_bar(acc));
+      }
+      if (signaler) {
+        volatile int never = 0;
+        // all eight epilogue warps of this CTA have stored this item
+        if (mbar_wait_bounded(epi_bar(acc), aph, abort_flag)) {
+          __threadfence();
+          red_release_gpu_add(done_counter(p, tl.mat, item.k, item.mode), 1);
+        } else {
+          fail(kErrTimeoutEpilogue);
+        }
+        (void)never;
+      }
+      __syncwarp();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  cluster_sync_all();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc_pair(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace muonb200

@@ -20,7 +20,7 @@
 #include "muon_b200.h"
 
 #include "k_ema.cuh"
-#include "k_ns_gemm.cuh"
+#include "k_ns_mega.cuh"
 #include "k_prologue.cuh"
 #include "muon_types.cuh"
 
@@ -28,10 +28,6 @@ using namespace muonb200;
 
 namespace {
 
-constexpr int kGramStages = 6;
-constexpr int kApplyStages = 4;
-using GramCfg = NsCfg<kGramN, false, kGramStages>;
-using ApplyCfg = NsCfg<kApplyN, true, kApplyStages>;
 constexpr int kMaxNsSteps = 16;
 constexpr int kMaxMats = 4096;
 constexpr int kMaxLaunchesPerStep = 1 + 3 * kMaxNsSteps;
@@ -85,6 +81,7 @@ struct Geom {
   int rows, cols, m, n, ldx, lda, transposed;
   size_t x_off[2], a_off, b_off;
   int part_first, part_count;
+  int n_sym_tiles, n_apply_tiles;
 };
 
 struct TimingSlot {
@@ -109,7 +106,9 @@ struct muon_plan {
   std::vector<NsTile> gram, poly, apply;
   size_t ws_bytes = 0;
   size_t part_off = 0;
+  size_t done_off = 0;
   size_t pro_smem = 0;
+  int max_clusters = 0;
 
   // device table: [MatDev x n_mats][ProItem][gram][poly][apply][err]
   void* d_block = nullptr;
@@ -197,6 +196,7 @@ struct LaunchTables {
   int32_t* err;
   int num_sms;
   size_t pro_smem;
+  int max_clusters;   // co-resident clusters of the Newton-Schulz kernel
 };
 
 muon_status_t validate_hyper(const muon_hyper_t* hyper, const float* ns_coeffs,
@@ -249,6 +249,8 @@ bool fill_workspace_fields(MatDev& d, const Geom& g, char* ws) {
   d.transposed = g.transposed;
   d.part_first = g.part_first;
   d.part_count = g.part_count;
+  d.n_sym_tiles = g.n_sym_tiles;
+  d.n_apply_tiles = g.n_apply_tiles;
   return true;
 }
 
@@ -266,10 +268,66 @@ bool fill_caller_fields(MatDev& d, const muon_matrix_t& mt) {
   return true;
 }
 
+// Clusters of two that can be resident at once (the persistent schedule
+// relies on every launched cluster being resident); 0 on failure.
+int query_max_clusters() {
+  if (cudaFuncSetAttribute(ns_mega_pair_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kMegaSmemBytes)) != cudaSuccess)
+    return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(kNsThreads);
+  cfg.dynamicSmemBytes = kMegaSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, ns_mega_pair_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+
+// Pair tiles of one matrix: symmetric products over upper 256 x 256 blocks,
+// the apply over all 256 x 256 blocks of X.  Returns false on overflow.
+bool append_pair_tiles(int mat, const Geom& g, NsTile* gram, NsTile* poly,
+                       int& n_gram, int cap_gram, NsTile* apply, int& n_apply,
+                       int cap_apply) {
+  const int t2 = ceil_div(g.m, kPairTile);
+  for (int ti = 0; ti < t2; ++ti)
+    for (int tj = ti; tj < t2; ++tj) {
+      if (n_gram >= cap_gram) return false;
+      gram[n_gram] = NsTile{static_cast<uint16_t>(mat), static_cast<uint16_t>(ti),
+                            static_cast<uint16_t>(tj),
+                            static_cast<uint16_t>(ceil_div(g.n, kTileK))};
+      poly[n_gram] = NsTile{static_cast<uint16_t>(mat), static_cast<uint16_t>(ti),
+                            static_cast<uint16_t>(tj),
+                            static_cast<uint16_t>(ceil_div(g.m, kTileK))};
+      ++n_gram;
+    }
+  const int tn = ceil_div(g.n, kPairTile);
+  for (int ti = 0; ti < t2; ++ti)
+    for (int tj = 0; tj < tn; ++tj) {
+      if (n_apply >= cap_apply) return false;
+      apply[n_apply++] = NsTile{static_cast<uint16_t>(mat), static_cast<uint16_t>(ti),
+                                static_cast<uint16_t>(tj),
+                                static_cast<uint16_t>(ceil_div(g.m, kTileK))};
+    }
+  return true;
+}
+
 // prologue -> K x (gram -> poly -> apply), or prologue -> final for K = 0.
 void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
                   const float* ns_coeffs, int32_t ns_steps, float* partials,
-                  int fault, bool fresh, cudaStream_t st, Recorder* rec) {
+                  int32_t* done, int done_count, int fault, bool fresh,
+                  cudaStream_t st, Recorder* rec) {
   HyperDev hd{h.momentum, h.lr, h.weight_decay, h.eps_row, h.eps_frob,
               h.nesterov, h.eq_r};
   muon_prologue_kernel<<<static_cast<unsigned>(t.n_items), kProThreads,
@@ -282,47 +340,48 @@ void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
                                      h.weight_decay, h.eps_frob);
     if (rec) rec->after(MUON_KIND_FINAL);
   }
-  for (int k = 0; k < ns_steps; ++k) {
-    NsParams p{};
+  if (ns_steps > 0) {
+    MegaParams p{};
     p.mats = t.mats;
+    p.gram = t.gram;
+    p.poly = t.poly;
+    p.apply = t.apply;
     p.partials = partials;
     p.err = t.err;
-    p.src = k & 1;
+    p.done = done;
+    p.n_gram = t.n_gram;
+    p.n_poly = t.n_poly;
+    p.n_apply = t.n_apply;
+    p.steps = ns_steps;
     p.fault = fault;
     p.fresh = fresh ? 1 : 0;
-    p.a = ns_coeffs[3 * k + 0];
-    p.b = ns_coeffs[3 * k + 1];
-    p.c = ns_coeffs[3 * k + 2];
+    for (int k = 0; k < ns_steps; ++k) {
+      p.a[k] = ns_coeffs[3 * k + 0];
+      p.b[k] = ns_coeffs[3 * k + 1];
+      p.c[k] = ns_coeffs[3 * k + 2];
+    }
     p.lr = h.lr;
     p.wd = h.weight_decay;
     p.eps_frob = h.eps_frob;
-
-    p.tiles = t.gram;
-    p.n_tiles = t.n_gram;
-    p.mode = kModeGram;
-    p.first = k == 0;
-    p.last = 0;
-    ns_gemm_kernel<kGramN, false, kGramStages>
-        <<<std::min(p.n_tiles, t.num_sms), kNsThreads, GramCfg::kSmemBytes, st>>>(p);
-    if (rec) rec->after(MUON_KIND_GRAM);
-
-    p.tiles = t.poly;
-    p.n_tiles = t.n_poly;
-    p.mode = kModePoly;
-    p.first = 0;
-    p.fault = 0;
-    ns_gemm_kernel<kGramN, false, kGramStages>
-        <<<std::min(p.n_tiles, t.num_sms), kNsThreads, GramCfg::kSmemBytes, st>>>(p);
-    if (rec) rec->after(MUON_KIND_POLY);
-
-    p.tiles = t.apply;
-    p.n_tiles = t.n_apply;
-    p.mode = kModeApply;
-    p.first = k == 0;
-    p.last = k == ns_steps - 1;
-    ns_gemm_kernel<kApplyN, true, kApplyStages>
-        <<<std::min(p.n_tiles, t.num_sms), kNsThreads, ApplyCfg::kSmemBytes, st>>>(p);
-    if (rec) rec->after(MUON_KIND_APPLY);
+    cudaMemsetAsync(done, 0, static_cast<size_t>(done_count) * sizeof(int32_t), st);
+    const long long items =
+        static_cast<long long>(ns_steps) * (t.n_gram + t.n_poly + t.n_apply);
+    const int clusters =
+        static_cast<int>(std::max<long long>(1, std::min<long long>(t.max_clusters, items)));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters);
+    cfg.blockDim = dim3(kNsThreads);
+    cfg.dynamicSmemBytes = kMegaSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, ns_mega_pair_kernel, p);
+    if (rec) rec->after(MUON_KIND_NS);
   }
 }
 
@@ -346,8 +405,9 @@ const char* muon_status_string(muon_status_t s) {
 }
 
 int32_t muon_step_launches(int32_t ns_steps) {
-  if (ns_steps < 0) return 0;
-  return ns_steps == 0 ? 2 : 1 + 3 * ns_steps;
+  // prologue, then one Newton-Schulz launch for all steps (or the K = 0
+  // finisher); the counter reset is a memset, not a kernel
+  return ns_steps < 0 ? 0 : 2;
 }
 
 int32_t ema_update_launches(int32_t n_tensors) {
@@ -412,22 +472,18 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
       plan->pro_smem = std::max(plan->pro_smem,
                                 static_cast<size_t>(rt) * (g.cols + 2) * 2);
 
-    const int tm = ceil_div(g.m, kTileM);
-    for (int ti = 0; ti < tm; ++ti)
-      for (int tj = ti; tj < tm; ++tj) {
-        plan->gram.push_back(NsTile{static_cast<uint16_t>(i), static_cast<uint16_t>(ti),
-                                    static_cast<uint16_t>(tj),
-                                    static_cast<uint16_t>(ceil_div(g.n, kTileK))});
-        plan->poly.push_back(NsTile{static_cast<uint16_t>(i), static_cast<uint16_t>(ti),
-                                    static_cast<uint16_t>(tj),
-                                    static_cast<uint16_t>(ceil_div(g.m, kTileK))});
-      }
-    const int tn = ceil_div(g.n, kApplyN);
-    for (int ti = 0; ti < tm; ++ti)
-      for (int tj = 0; tj < tn; ++tj)
-        plan->apply.push_back(NsTile{static_cast<uint16_t>(i), static_cast<uint16_t>(ti),
-                                     static_cast<uint16_t>(tj),
-                                     static_cast<uint16_t>(ceil_div(g.m, kTileK))});
+    {
+      const int t2 = ceil_div(g.m, kPairTile), tn = ceil_div(g.n, kPairTile);
+      const size_t ng = plan->gram.size(), na = plan->apply.size();
+      plan->gram.resize(ng + t2 * (t2 + 1) / 2);
+      plan->poly.resize(ng + t2 * (t2 + 1) / 2);
+      plan->apply.resize(na + static_cast<size_t>(t2) * tn);
+      int n_gram = 0, n_apply = 0;
+      append_pair_tiles(i, g, plan->gram.data() + ng, plan->poly.data() + ng, n_gram,
+                        t2 * (t2 + 1) / 2, plan->apply.data() + na, n_apply, t2 * tn);
+      g.n_sym_tiles = n_gram;
+      g.n_apply_tiles = n_apply;
+    }
   }
   if (plan->items.size() > 0x7FFFFFFF ||
       plan->gram.size() > 0x7FFFFFFF || plan->apply.size() > 0x7FFFFFFF) {
@@ -439,6 +495,9 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
   sort_tiles(plan->apply);
   plan->part_off = off;
   off = align_up(off + plan->items.size() * sizeof(float), 1024);
+  plan->done_off = off;
+  off = align_up(off + static_cast<size_t>(n_mats) * std::max(max_ns_steps, 1) * 3 *
+                           sizeof(int32_t), 1024);
   plan->ws_bytes = off;
 
   // Device table.
@@ -478,12 +537,7 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
                  cudaMemcpyHostToDevice) == cudaSuccess &&
       cudaMemset(plan->d_err, 0, sizeof(int32_t)) == cudaSuccess;
   ok = ok &&
-       cudaFuncSetAttribute(ns_gemm_kernel<kGramN, false, kGramStages>,
-                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                            static_cast<int>(GramCfg::kSmemBytes)) == cudaSuccess &&
-       cudaFuncSetAttribute(ns_gemm_kernel<kApplyN, true, kApplyStages>,
-                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                            static_cast<int>(ApplyCfg::kSmemBytes)) == cudaSuccess &&
+       (plan->max_clusters = query_max_clusters()) > 0 &&
        cudaFuncSetAttribute(muon_prologue_kernel,
                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                             static_cast<int>(std::max<size_t>(plan->pro_smem, 1024))) ==
@@ -621,11 +675,12 @@ muon_status_t muon_step_batched(muon_plan_t* plan, const muon_matrix_t* mats,
                  plan->d_gram, static_cast<int>(plan->gram.size()),
                  plan->d_poly, static_cast<int>(plan->poly.size()),
                  plan->d_apply, static_cast<int>(plan->apply.size()),
-                 plan->d_err, plan->num_sms, plan->pro_smem};
+                 plan->d_err, plan->num_sms, plan->pro_smem, plan->max_clusters};
   float* partials = reinterpret_cast<float*>(ws + plan->part_off);
+  int32_t* done = reinterpret_cast<int32_t*>(ws + plan->done_off);
   Recorder rec(plan, st);
-  enqueue_step(t, *hyper, ns_coeffs, ns_steps, partials, plan->fault, changed, st,
-               plan->timing ? &rec : nullptr);
+  enqueue_step(t, *hyper, ns_coeffs, ns_steps, partials, done, plan->n_mats * ns_steps * 3,
+               plan->fault, changed, st, plan->timing ? &rec : nullptr);
   rec.finish();
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
@@ -706,6 +761,7 @@ constexpr int kNoAllocMaxApplyTiles = 8192;
 
 // Device address of g_noalloc_scratch per device (filled on first use).
 void* g_noalloc_dev_ptr[kNoAllocMaxDevices] = {};
+int g_noalloc_clusters[kNoAllocMaxDevices] = {};
 std::mutex g_noalloc_mutex;
 
 // Host-side staging of the tables (fixed capacity; guarded by the mutex).
@@ -791,32 +847,21 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
     if (g.transposed)
       pro_smem = std::max(pro_smem, static_cast<size_t>(rt) * (g.cols + 2) * 2);
 
-    const int tm = ceil_div(g.m, kTileM);
-    for (int ti = 0; ti < tm; ++ti)
-      for (int tj = ti; tj < tm; ++tj) {
-        if (n_gram >= kNoAllocMaxGramTiles) return MUON_ERR_UNSUPPORTED;
-        g_na_gram[n_gram] = NsTile{static_cast<uint16_t>(i), static_cast<uint16_t>(ti),
-                                   static_cast<uint16_t>(tj),
-                                   static_cast<uint16_t>(ceil_div(g.n, kTileK))};
-        g_na_poly[n_gram] = NsTile{static_cast<uint16_t>(i), static_cast<uint16_t>(ti),
-                                   static_cast<uint16_t>(tj),
-                                   static_cast<uint16_t>(ceil_div(g.m, kTileK))};
-        ++n_gram;
-      }
-    const int tn = ceil_div(g.n, kApplyN);
-    for (int ti = 0; ti < tm; ++ti)
-      for (int tj = 0; tj < tn; ++tj) {
-        if (n_apply >= kNoAllocMaxApplyTiles) return MUON_ERR_UNSUPPORTED;
-        g_na_apply[n_apply++] = NsTile{static_cast<uint16_t>(i), static_cast<uint16_t>(ti),
-                                       static_cast<uint16_t>(tj),
-                                       static_cast<uint16_t>(ceil_div(g.m, kTileK))};
-      }
+    const int gram_before = n_gram, apply_before = n_apply;
+    if (!append_pair_tiles(i, g, g_na_gram, g_na_poly, n_gram, kNoAllocMaxGramTiles,
+                           g_na_apply, n_apply, kNoAllocMaxApplyTiles))
+      return MUON_ERR_UNSUPPORTED;
+    g.n_sym_tiles = n_gram - gram_before;
+    g.n_apply_tiles = n_apply - apply_before;
   }
   sort_tiles_by_k(g_na_gram, n_gram);
   sort_tiles_by_k(g_na_poly, n_gram);
   sort_tiles_by_k(g_na_apply, n_apply);
   const size_t part_off = off;
   off = align_up(off + static_cast<size_t>(n_items) * sizeof(float), 1024);
+  const size_t done_off = off;
+  off = align_up(off + static_cast<size_t>(n_mats) * std::max(ns_steps, 1) * 3 *
+                           sizeof(int32_t), 1024);
   const size_t ws_bytes = off;
 
   // Layout of the device array: [error word][tables][workspace].
@@ -844,15 +889,12 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
       cudaGetLastError();
       return MUON_ERR_CUDA;
     }
-    if (cudaFuncSetAttribute(ns_gemm_kernel<kGramN, false, kGramStages>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(GramCfg::kSmemBytes)) != cudaSuccess ||
-        cudaFuncSetAttribute(ns_gemm_kernel<kApplyN, true, kApplyStages>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(ApplyCfg::kSmemBytes)) != cudaSuccess) {
+    const int clusters = query_max_clusters();
+    if (clusters <= 0) {
       cudaGetLastError();
       return MUON_ERR_CUDA;
     }
+    g_noalloc_clusters[dev] = clusters;
     g_noalloc_dev_ptr[dev] = ptr;
   }
   int num_sms = 148;
@@ -896,9 +938,12 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
                  reinterpret_cast<const NsTile*>(base + gram_off), n_gram,
                  reinterpret_cast<const NsTile*>(base + poly_off), n_gram,
                  reinterpret_cast<const NsTile*>(base + apply_off), n_apply,
-                 reinterpret_cast<int32_t*>(base), num_sms, pro_smem};
+                 reinterpret_cast<int32_t*>(base), num_sms, pro_smem,
+                 g_noalloc_clusters[dev]};
   float* partials = reinterpret_cast<float*>(ws + part_off);
-  enqueue_step(t, *hyper, ns_coeffs, ns_steps, partials, 0, true, st, nullptr);
+  int32_t* done = reinterpret_cast<int32_t*>(ws + done_off);
+  enqueue_step(t, *hyper, ns_coeffs, ns_steps, partials, done, n_mats * ns_steps * 3, 0,
+               true, st, nullptr);
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
 }

@@ -7,10 +7,8 @@
 
 namespace muonb200 {
 
-constexpr int kTileM = 128;       // UMMA M (rows of a tile)
+constexpr int kTileM = 128;       // rows of a tile held by one CTA (TMEM lanes)
 constexpr int kTileK = 64;        // K per pipeline stage (one 128-B swizzle row)
-constexpr int kGramN = 128;       // square tiles for the symmetric products
-constexpr int kApplyN = 256;      // wide tiles for X <- a X + B X
 constexpr int kProRows = 32;      // rows per prologue work item
 constexpr int kProThreads = 256;  // 8 warps
 constexpr int kProCachedChunks = 8;  // row chunks (of 256 elements) kept in
@@ -35,6 +33,8 @@ struct alignas(64) MatDev {
   int32_t transposed;    // rows > cols
   int32_t part_first;    // first prologue partial of this matrix
   int32_t part_count;    // number of prologue partials
+  int32_t n_sym_tiles;   // 256 x 256 pair tiles of A (and of B'), upper blocks
+  int32_t n_apply_tiles; // 256 x 256 pair tiles of X
   float update_scale;
 };
 
@@ -61,21 +61,6 @@ struct HyperDev {
 
 enum NsMode : int32_t { kModeGram = 0, kModePoly = 1, kModeApply = 2 };
 
-struct NsParams {
-  const MatDev* mats;
-  const NsTile* tiles;
-  const float* partials;
-  int32_t* err;
-  int32_t n_tiles;
-  int32_t mode;
-  int32_t src;     // X buffer holding the current X
-  int32_t first;   // Newton-Schulz step 0: fold the Frobenius scale
-  int32_t last;    // last step: write W (and O) instead of X
-  int32_t fault;   // test hook (see muon_plan_set_fault)
-  int32_t fresh;   // the tensor maps were (re)written before this step
-  float a, b, c;
-  float lr, wd, eps_frob;
-};
 
 // Error word values (device -> host).
 constexpr int32_t kErrTimeoutProducer = 0x101;

@@ -1,0 +1,107 @@
+"""Multi-process host logic on CPU (gloo, world size 2): matrix ownership,
+the reduce / step / broadcast exchange of a sharded step, and the benchmark's
+max-over-ranks timing.  The per-rank compute is the fp64 oracle here; on GPUs
+it is the library's step."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from muon_optimizer_step_02_b200 import sharding, workloads as wl
+
+
+def test_partition_is_balanced_and_complete():
+    shapes = wl.workload(2).shapes
+    for world in (1, 2, 4, 8):
+        owner = sharding.partition_matrices(shapes, world)
+        assert len(owner) == len(shapes)
+        assert set(owner) <= set(range(world))
+        loads = sharding.rank_loads(shapes, owner, world)
+        total = sum(loads)
+        biggest = max(sharding.matrix_cost(r, c, 5) for r, c in shapes)
+        # LPT bound: max load <= total/world + largest item
+        assert max(loads) <= total / world + biggest + 1e-6
+        assert owner == sharding.partition_matrices(shapes, world)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    import oracle.muon_oracle as mo
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            init_method=f"tcp://127.0.0.1:{port}")
+    try:
+        shapes = [(48, 32), (32, 48), (40, 40), (16, 64), (64, 16), (24, 24)]
+        h = wl.Hyper(momentum=0.9, lr=0.05, weight_decay=0.1)
+        coeffs = [wl.FIXED_QUINTIC] * 3
+        w = wl.custom(shapes, h, coeffs, grad_std=1.0, wid=400)
+        owner = sharding.partition_matrices(shapes, world, 3)
+        W = [torch.from_numpy(wl.weight(w, i).astype(np.float64))
+             for i in range(len(shapes))]
+        M = [torch.zeros_like(x) for x in W]
+        hyp = mo.MuonHyper(momentum=h.momentum, lr=h.lr,
+                           weight_decay=h.weight_decay)
+        for step in range(2):
+            # rank r holds a share of the gradient: the shares sum to G
+            G = [wl.bf16_bits_to_f32(wl.grad_bits(w, i, step)).astype(np.float64)
+                 for i in range(len(shapes))]
+            G_local = [torch.from_numpy(g * (0.25 if rank == 0 else 0.75))
+                       for g in G]
+
+            def step_fn(idx):
+                for i in idx:
+                    Wn, Mn, _ = mo.muon_step(W[i].numpy(), M[i].numpy(),
+                                             G_local[i].numpy(), hyp, coeffs,
+                                             1.0)
+                    W[i].copy_(torch.from_numpy(Wn))
+                    M[i].copy_(torch.from_numpy(Mn))
+
+            sharding.sharded_step(W, M, G_local, owner, rank, step_fn)
+        t = sharding.max_over_ranks(1.0 + rank)
+        q.put((rank, [x.numpy().copy() for x in W], t))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_step_matches_single_process():
+    import oracle.muon_oracle as mo
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    # single-process reference
+    shapes = [(48, 32), (32, 48), (40, 40), (16, 64), (64, 16), (24, 24)]
+    h = wl.Hyper(momentum=0.9, lr=0.05, weight_decay=0.1)
+    coeffs = [wl.FIXED_QUINTIC] * 3
+    w = wl.custom(shapes, h, coeffs, grad_std=1.0, wid=400)
+    hyp = mo.MuonHyper(momentum=h.momentum, lr=h.lr, weight_decay=h.weight_decay)
+    W = [wl.weight(w, i).astype(np.float64) for i in range(len(shapes))]
+    M = [np.zeros_like(x) for x in W]
+    for step in range(2):
+        for i in range(len(shapes)):
+            G = wl.bf16_bits_to_f32(wl.grad_bits(w, i, step)).astype(np.float64)
+            W[i], M[i], _ = mo.muon_step(W[i], M[i], G, hyp, coeffs, 1.0)
+    for rank, Ws, t in out:
+        assert t == 2.0            # max over ranks of 1.0 + rank
+        for a, b in zip(Ws, W):
+            np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
