@@ -43,7 +43,6 @@
 #include <cuda_bf16.h>
 
 #include "k_ns_common.cuh"
-#include "k_ns_gemm_pair.cuh"
 #include "muon_types.cuh"
 #include "sm100_ptx.cuh"
 
@@ -57,7 +56,7 @@ struct MegaParams {
   const NsTile* gram;     // pair tiles, K = n
   const NsTile* poly;     // pair tiles, K = m
   const NsTile* apply;    // pair tiles, K = m
-  const float* partials;
+  const float* mat_scale; // per-matrix Frobenius scale from the prologue
   int32_t* err;
   int32_t* done;          // [mat][step][phase] completion counts, zeroed
   int32_t n_gram, n_poly, n_apply;
@@ -67,9 +66,24 @@ struct MegaParams {
   float lr, wd, eps_frob;
 };
 
-using MegaCfg = PairCfg<false, kMegaStages>;   // 32 KB stages + transpose buffers
-// two more barriers than PairCfg (the epilogue completion pair), plus slack
-constexpr size_t kMegaSmemBytes = MegaCfg::kSmemBytes + 64;
+// Shared memory: the operand ring (per stage 16 KB of A rows + 16 KB of B
+// columns), then per epilogue warp a 32 x 32 bf16 output block and its
+// transpose (TMA-store sources), then the barriers.
+struct MegaCfg {
+  static constexpr int kABytes = 128 * kTileK * 2;
+  static constexpr int kBBytes = (kPairTile / 2) * kTileK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr uint32_t kTxBytes = 2u * kStageBytes;   // both CTAs
+  static constexpr int kTmemCols = 2 * kPairTile;
+  static constexpr int kOutBlockElems = 32 * 32;
+  static constexpr int kOutStageBytes = kEpiWarps * 2 * kOutBlockElems * 2;
+  static constexpr int kNumBars = 2 * kMegaStages + 7;
+  static constexpr size_t kSmemBytes = 1024 +
+      static_cast<size_t>(kMegaStages) * kStageBytes + kOutStageBytes +
+      kNumBars * 8 + 16;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+constexpr size_t kMegaSmemBytes = MegaCfg::kSmemBytes;
 
 // Spins (acquire) until *ctr >= target.  Gives up on the CTA's abort flag,
 // on a non-zero global error word (another CTA failed) or after the limit.
@@ -139,12 +153,12 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __nv_bfloat16* xpose =
+  __nv_bfloat16* out_stage =
       reinterpret_cast<__nv_bfloat16*>(smem + kMegaStages * Cfg::kStageBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(
-      smem + kMegaStages * Cfg::kStageBytes + Cfg::kXposeBytes);
+      smem + kMegaStages * Cfg::kStageBytes + Cfg::kOutStageBytes);
   // bars: full[S], empty[S], tfull[2], tempty[2], drain, epi[2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::kNumBars + 2);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   constexpr int S = kMegaStages;
 
@@ -319,7 +333,38 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
     const int quad = warp & 3;
     const int half = ew >> 2;
     const int r_pair = static_cast<int>(rank) * 128 + quad * 32 + lane;
-    __nv_bfloat16* xbuf = xpose + ew * 32 * kXposeLd;
+    // This warp's 32 x 32 output block (row = lane) and its transpose.
+    __nv_bfloat16* stg_d = out_stage + ew * 2 * Cfg::kOutBlockElems;
+    __nv_bfloat16* stg_m = stg_d + Cfg::kOutBlockElems;
+    const uint32_t stg_d_addr = smem_addr(stg_d);
+    const uint32_t stg_m_addr = smem_addr(stg_m);
+    // Stages v (row `lane`) into the direct block and, if asked, the
+    // transposed block, then one lane issues the TMA stores.
+    auto put_block = [&](const CUtensorMap* tm, int row0_, int col0_, bool mirror,
+                         const float (&v)[32]) {
+      if (lane == 0) bulk_wait_group_read0();   // previous blocks read out
+      __syncwarp();
+      uint4* drow = reinterpret_cast<uint4*>(stg_d + lane * 32);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        __nv_bfloat162 h[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          h[i] = __floats2bfloat162_rn(v[8 * q + 2 * i], v[8 * q + 2 * i + 1]);
+        drow[q] = *reinterpret_cast<uint4*>(h);
+      }
+      if (mirror) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) stg_m[e * 32 + lane] = __float2bfloat16_rn(v[e]);
+      }
+      fence_proxy_async_shared();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(tm, stg_d_addr, col0_, row0_);
+        if (mirror) tma_store_2d(tm, stg_m_addr, row0_, col0_);
+        bulk_commit_group();
+      }
+    };
     const uint32_t leader_tempty0 = mapa_shared(tempty_bar(0), 0);
     const bool signaler = ew == 0 && lane == 0;
     int lt = 0;
@@ -342,10 +387,9 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
       const bool row_ok = row < m;
       const bool first = item.k == 0;
       const bool last = item.k == p.steps - 1;
-      const float s = first ? frob_scale(md, p.partials, p.eps_frob) : 1.f;
+      const float s = first ? p.mat_scale[tl.mat] : 1.f;
 
       if (item.mode == kModeGram || item.mode == kModePoly) {
-        __nv_bfloat16* outp = (item.mode == kModeGram) ? md->a : md->b;
         const bool diag_tile = tl.ti == tl.tj;
         if (item.mode == kModePoly) {
           // The generic reads of A below need the gram stores of other CTAs.
@@ -379,14 +423,11 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
                 if (e == d) v[e] += pa;
             }
           }
-          if (row_ok)
-            store_row32_bf16(outp + static_cast<size_t>(row) * md->lda, col0, m, v);
-          if (!diag_tile)
-            store_mirror32_bf16(outp, md->lda, row0, col0, m, lane, xbuf, v);
+          put_block(item.mode == kModeGram ? &md->tm_as : &md->tm_bs, row0, col0,
+                    !diag_tile, v);
         }
       } else {
         const int n = md->n;
-        __nv_bfloat16* xd = md->x[(item.k & 1) ^ 1] + static_cast<size_t>(row) * md->ldx;
         const float decay = 1.f - p.lr * p.wd;
         const float step = p.lr * md->update_scale;
         const bool tr = md->transposed != 0;
@@ -420,15 +461,17 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
           }
           float v[32];
           tmem_load_32cols(tbase + cc * 32, v);
-          if (!live) continue;
           if (first) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] *= s;
           }
           if (!last) {
-            store_row32_bf16(xd, col0, n, v);
+            // rows beyond m and columns beyond n are clipped by the TMA store
+            if (row0 < m && col0 < n)
+              put_block(&md->tm_xs[(item.k & 1) ^ 1], row0, col0, false, v);
             continue;
           }
+          if (!live) continue;
 #pragma unroll
           for (int e = 0; e < 32; ++e) wv[e] = fmaf(wv[e], decay, -step * v[e]);
           if (!tr) {
@@ -463,7 +506,9 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
       }
       // Accumulator free: the leader may start the item after next.
       tc_fence_before();
-      // Outputs of this item visible (to TMA readers too) before counting it.
+      // This warp's stores of the item complete and visible (TMA readers
+      // too) before the item is counted.
+      if (lane == 0) bulk_wait_group0();
       fence_proxy_async_global();
       __syncwarp();
       if (lane == 0) {

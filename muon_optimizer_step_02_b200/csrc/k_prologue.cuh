@@ -5,6 +5,10 @@
 // working orientation (transposed through shared memory when rows > cols);
 // the Frobenius partial sum of X~ over the work item goes to `partials`.
 //
+// The Frobenius scale s = 1 / (||X~||_F + eps_frob) of each matrix is also
+// finished here: every block writes its partial sum, and the last block of a
+// matrix (ticket counter) adds the matrix's partials in index order.
+//
 // Sources: PR #1893 "Record: L_ParallelResiduals_UNetSkips_DepthRecur_Muon_
 // 1.0901", table "Architecture and training stack", row "Optimizer" (Muon,
 // momentum 0.99); PR #1396 "Record: Combined 3-Layer Recurrence + Parallel
@@ -41,9 +45,9 @@ __device__ __forceinline__ void load_g_m(const uint16_t* __restrict__ g,
   if (vec) {
     const int p0 = ch * 256 + lane * 8;
     if (p0 < cols) {
-      const uint4 graw = __ldcs(reinterpret_cast<const uint4*>(g + p0));
-      const float4 m0 = __ldcs(reinterpret_cast<const float4*>(mo + p0));
-      const float4 m1 = __ldcs(reinterpret_cast<const float4*>(mo + p0 + 4));
+      const uint4 graw = *reinterpret_cast<const uint4*>(g + p0);
+      const float4 m0 = *reinterpret_cast<const float4*>(mo + p0);
+      const float4 m1 = *reinterpret_cast<const float4*>(mo + p0 + 4);
       const uint32_t gw[4] = {graw.x, graw.y, graw.z, graw.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -72,10 +76,9 @@ __device__ __forceinline__ void store_m(float* __restrict__ mo, bool vec,
   if (vec) {
     const int p0 = ch * 256 + lane * 8;
     if (p0 < cols) {
-      __stcs(reinterpret_cast<float4*>(mo + p0),
-             make_float4(mv[0], mv[1], mv[2], mv[3]));
-      __stcs(reinterpret_cast<float4*>(mo + p0 + 4),
-             make_float4(mv[4], mv[5], mv[6], mv[7]));
+      // default caching: pass 2 re-reads M' from L2
+      *reinterpret_cast<float4*>(mo + p0) = make_float4(mv[0], mv[1], mv[2], mv[3]);
+      *reinterpret_cast<float4*>(mo + p0 + 4) = make_float4(mv[4], mv[5], mv[6], mv[7]);
     }
   } else {
 #pragma unroll
@@ -119,12 +122,46 @@ __device__ __forceinline__ void emit_x(__nv_bfloat16* __restrict__ xrow,
   }
 }
 
-__global__ void __launch_bounds__(kProThreads)
+// Loads of one chunk kept raw: G as 8 packed bf16, M as 8 floats.
+struct ChunkRaw {
+  uint4 g;
+  float4 m0, m1;
+};
+
+__device__ __forceinline__ void load_chunk_vec(const uint16_t* __restrict__ g,
+                                               const float* __restrict__ mo,
+                                               int p0, ChunkRaw& c) {
+  c.g = *reinterpret_cast<const uint4*>(g + p0);
+  c.m0 = *reinterpret_cast<const float4*>(mo + p0);
+  c.m1 = *reinterpret_cast<const float4*>(mo + p0 + 4);
+}
+
+__device__ __forceinline__ void unpack_chunk(const ChunkRaw& c, float (&gv)[8],
+                                             float (&mv)[8]) {
+  const uint32_t gw[4] = {c.g.x, c.g.y, c.g.z, c.g.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    gv[2 * i] = __uint_as_float(gw[i] << 16);
+    gv[2 * i + 1] = __uint_as_float(gw[i] & 0xFFFF0000u);
+  }
+  mv[0] = c.m0.x; mv[1] = c.m0.y; mv[2] = c.m0.z; mv[3] = c.m0.w;
+  mv[4] = c.m1.x; mv[5] = c.m1.y; mv[6] = c.m1.z; mv[7] = c.m1.w;
+}
+
+// One warp per stored row, two passes over the row with no register copy of
+// it: pass 1 streams G and M (kProBatch chunks of 8 elements per lane in
+// flight), writes M' and sums U^2; pass 2 re-reads G and the M' it just wrote
+// (L2-resident), rebuilds U and writes the normalised row.  Keeping the row
+// out of registers keeps occupancy at three blocks (24 warps) per SM with
+// two chunks in flight per lane.
+__global__ void __launch_bounds__(kProThreads, 3)
 muon_prologue_kernel(const MatDev* __restrict__ mats,
                      const ProItem* __restrict__ items, HyperDev h,
-                     float* __restrict__ partials) {
+                     float* __restrict__ partials, int32_t* __restrict__ tickets,
+                     float* __restrict__ mat_scale) {
   extern __shared__ __align__(16) unsigned char pro_smem[];
   __shared__ float warp_sums[kProThreads / 32];
+  __shared__ int last_block;
 
   const ProItem it = items[blockIdx.x];
   const MatDev& md = mats[it.mat];
@@ -141,67 +178,92 @@ muon_prologue_kernel(const MatDev* __restrict__ mats,
   for (int r = warp; r < it.nrows; r += kProThreads / 32) {
     const int row = it.row0 + r;
     const size_t base = static_cast<size_t>(row) * cols;
-    const uint16_t* g = md.g + base;
-    float* mo = md.mom + base;
+    const uint16_t* __restrict__ g = md.g + base;
+    float* __restrict__ mo = md.mom + base;
     __nv_bfloat16* xrow = tr ? nullptr : md.x[0] + static_cast<size_t>(row) * md.ldx;
     __nv_bfloat16* srow = tr ? stage + r * sld : nullptr;
 
-    float cache[kProCachedChunks][8];
+    // Pass 1: M' = mu M + G (stored), U = G + mu M', sum of U^2.
     float ss = 0.f;
-    // Pass 1: momentum update, look-ahead, row sum of squares.
+    for (int c0 = 0; c0 < nch; c0 += kProBatch) {
+      if (vec) {
+        ChunkRaw raw[kProBatch];
 #pragma unroll
-    for (int ch = 0; ch < kProCachedChunks; ++ch) {
-      if (ch < nch) {
-        float gv[8], mv[8];
-        load_g_m(g, mo, vec, ch, lane, cols, gv, mv);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float mn = fmaf(mu, mv[e], gv[e]);
-          const float u = h.nesterov ? fmaf(mu, mn, gv[e]) : mn;
-          mv[e] = mn;
-          cache[ch][e] = u;
-          ss = fmaf(u, u, ss);
+        for (int b = 0; b < kProBatch; ++b) {
+          const int p0 = (c0 + b) * 256 + lane * 8;
+          if (c0 + b < nch && p0 < cols) load_chunk_vec(g, mo, p0, raw[b]);
         }
-        store_m(mo, vec, ch, lane, cols, mv);
-      }
-    }
-    for (int ch = kProCachedChunks; ch < nch; ++ch) {
-      float gv[8], mv[8];
-      load_g_m(g, mo, vec, ch, lane, cols, gv, mv);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float mn = fmaf(mu, mv[e], gv[e]);
-        const float u = h.nesterov ? fmaf(mu, mn, gv[e]) : mn;
-        mv[e] = mn;
-        ss = fmaf(u, u, ss);
+        for (int b = 0; b < kProBatch; ++b) {
+          const int p0 = (c0 + b) * 256 + lane * 8;
+          if (c0 + b < nch && p0 < cols) {
+            float gv[8], mv[8];
+            unpack_chunk(raw[b], gv, mv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float mn = fmaf(mu, mv[e], gv[e]);
+              const float u = h.nesterov ? fmaf(mu, mn, gv[e]) : mn;
+              mv[e] = mn;
+              ss = fmaf(u, u, ss);
+            }
+            store_m(mo, true, c0 + b, lane, cols, mv);
+          }
+        }
+      } else {
+        for (int b = 0; b < kProBatch && c0 + b < nch; ++b) {
+          float gv[8], mv[8];
+          load_g_m(g, mo, false, c0 + b, lane, cols, gv, mv);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float mn = fmaf(mu, mv[e], gv[e]);
+            const float u = h.nesterov ? fmaf(mu, mn, gv[e]) : mn;
+            mv[e] = mn;
+            ss = fmaf(u, u, ss);
+          }
+          store_m(mo, false, c0 + b, lane, cols, mv);
+        }
       }
-      store_m(mo, vec, ch, lane, cols, mv);
     }
     ss = warp_allreduce_sum(ss);
     const float inv = h.eq_r ? 1.f / (sqrtf(ss) + h.eps_row) : 1.f;
     fro += ss * inv * inv;
+    __syncwarp();  // this lane's M' stores precede its own re-reads below
 
-    // Pass 2: normalised row in bf16.
+    // Pass 2: U again from G and M', normalised, bf16.
+    for (int c0 = 0; c0 < nch; c0 += kProBatch) {
+      if (vec) {
+        ChunkRaw raw[kProBatch];
 #pragma unroll
-    for (int ch = 0; ch < kProCachedChunks; ++ch) {
-      if (ch < nch) {
-        float x[8];
+        for (int b = 0; b < kProBatch; ++b) {
+          const int p0 = (c0 + b) * 256 + lane * 8;
+          if (c0 + b < nch && p0 < cols) load_chunk_vec(g, mo, p0, raw[b]);
+        }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = cache[ch][e] * inv;
-        emit_x(xrow, srow, tr, vec, ch, lane, cols, x);
+        for (int b = 0; b < kProBatch; ++b) {
+          const int p0 = (c0 + b) * 256 + lane * 8;
+          if (c0 + b < nch && p0 < cols) {
+            float gv[8], mv[8], x[8];
+            unpack_chunk(raw[b], gv, mv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float u = h.nesterov ? fmaf(mu, mv[e], gv[e]) : mv[e];
+              x[e] = u * inv;
+            }
+            emit_x(xrow, srow, tr, true, c0 + b, lane, cols, x);
+          }
+        }
+      } else {
+        for (int b = 0; b < kProBatch && c0 + b < nch; ++b) {
+          float gv[8], mv[8], x[8];
+          load_g_m(g, mo, false, c0 + b, lane, cols, gv, mv);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float u = h.nesterov ? fmaf(mu, mv[e], gv[e]) : mv[e];
+            x[e] = u * inv;
+          }
+          emit_x(xrow, srow, tr, false, c0 + b, lane, cols, x);
+        }
       }
-    }
-    for (int ch = kProCachedChunks; ch < nch; ++ch) {
-      // Rows longer than the register cache: recompute U from G and the
-      // momentum this thread has just written.
-      float gv[8], mv[8], x[8];
-      load_g_m(g, mo, vec, ch, lane, cols, gv, mv);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float u = h.nesterov ? fmaf(mu, mv[e], gv[e]) : mv[e];
-        x[e] = u * inv;
-      }
-      emit_x(xrow, srow, tr, vec, ch, lane, cols, x);
     }
   }
 
@@ -212,6 +274,21 @@ muon_prologue_kernel(const MatDev* __restrict__ mats,
 #pragma unroll
     for (int w = 0; w < kProThreads / 32; ++w) s += warp_sums[w];
     partials[blockIdx.x] = s;
+    // The last block of this matrix sums its partials in index order (the
+    // same order whichever block is last) into the Frobenius scale.
+    __threadfence();
+    const int ticket = atomicAdd(&tickets[it.mat], 1);
+    last_block = ticket == md.part_count - 1;
+  }
+  __syncthreads();
+  if (last_block && warp == 0) {
+    __threadfence();
+    float sum = 0.f;
+    if (lane == 0) {
+      const volatile float* pv = partials + md.part_first;
+      for (int i = 0; i < md.part_count; ++i) sum += pv[i];
+      mat_scale[it.mat] = 1.f / (sqrtf(sum) + h.eps_frob);
+    }
   }
 
   if (tr) {
@@ -241,13 +318,10 @@ muon_prologue_kernel(const MatDev* __restrict__ mats,
 __global__ void __launch_bounds__(kProThreads)
 muon_final_noiter_kernel(const MatDev* __restrict__ mats,
                          const ProItem* __restrict__ items,
-                         const float* __restrict__ partials, float lr, float wd,
-                         float eps_frob) {
+                         const float* __restrict__ mat_scale, float lr, float wd) {
   const ProItem it = items[blockIdx.x];
   const MatDev& md = mats[it.mat];
-  float sum = 0.f;
-  for (int i = 0; i < md.part_count; ++i) sum += partials[md.part_first + i];
-  const float s = 1.f / (sqrtf(sum) + eps_frob);
+  const float s = mat_scale[it.mat];
   const float decay = 1.f - lr * wd;
   const float step = lr * md.update_scale;
   const int cols = md.cols;

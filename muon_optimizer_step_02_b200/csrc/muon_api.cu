@@ -32,7 +32,7 @@ constexpr int kMaxNsSteps = 16;
 constexpr int kMaxMats = 4096;
 constexpr int kMaxLaunchesPerStep = 1 + 3 * kMaxNsSteps;
 constexpr int kTimingSlots = 64;
-constexpr size_t kProSmemCap = 200 * 1024;
+constexpr size_t kProSmemCap = 48 * 1024;   // four prologue blocks per SM
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -60,9 +60,10 @@ EncodeTiledFn get_encode_fn() {
 }
 
 // bf16 matrix of `rows` x `cols` elements with leading dimension `ld`,
-// 128-byte swizzled boxes of box_cols x box_rows.
+// boxes of box_cols x box_rows (128-byte swizzle for operand loads, none for
+// the epilogue's 32 x 32 stores).
 bool encode_bf16_2d(CUtensorMap* tm, void* base, int rows, int cols, int ld,
-                    int box_cols, int box_rows) {
+                    int box_cols, int box_rows, bool swizzle = true) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols),
@@ -72,7 +73,8 @@ bool encode_bf16_2d(CUtensorMap* tm, void* base, int rows, int cols, int ld,
                        static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -106,7 +108,9 @@ struct muon_plan {
   std::vector<NsTile> gram, poly, apply;
   size_t ws_bytes = 0;
   size_t part_off = 0;
-  size_t done_off = 0;
+  size_t scale_off = 0;
+  size_t counter_off = 0;
+  size_t counter_bytes = 0;
   size_t pro_smem = 0;
   int max_clusters = 0;
 
@@ -232,13 +236,16 @@ bool fill_workspace_fields(MatDev& d, const Geom& g, char* ws) {
   for (int b = 0; b < 2; ++b) {
     d.x[b] = reinterpret_cast<__nv_bfloat16*>(ws + g.x_off[b]);
     if (!encode_bf16_2d(&d.tm_xk[b], d.x[b], g.m, g.n, g.ldx, kTileK, kTileM) ||
-        !encode_bf16_2d(&d.tm_xn[b], d.x[b], g.m, g.n, g.ldx, 64, kTileK))
+        !encode_bf16_2d(&d.tm_xn[b], d.x[b], g.m, g.n, g.ldx, 64, kTileK) ||
+        !encode_bf16_2d(&d.tm_xs[b], d.x[b], g.m, g.n, g.ldx, 32, 32, false))
       return false;
   }
   d.a = reinterpret_cast<__nv_bfloat16*>(ws + g.a_off);
   d.b = reinterpret_cast<__nv_bfloat16*>(ws + g.b_off);
   if (!encode_bf16_2d(&d.tm_a, d.a, g.m, g.m, g.lda, kTileK, kTileM) ||
-      !encode_bf16_2d(&d.tm_b, d.b, g.m, g.m, g.lda, kTileK, kTileM))
+      !encode_bf16_2d(&d.tm_b, d.b, g.m, g.m, g.lda, kTileK, kTileM) ||
+      !encode_bf16_2d(&d.tm_as, d.a, g.m, g.m, g.lda, 32, 32, false) ||
+      !encode_bf16_2d(&d.tm_bs, d.b, g.m, g.m, g.lda, 32, 32, false))
     return false;
   d.rows = g.rows;
   d.cols = g.cols;
@@ -324,20 +331,32 @@ bool append_pair_tiles(int mat, const Geom& g, NsTile* gram, NsTile* poly,
 }
 
 // prologue -> K x (gram -> poly -> apply), or prologue -> final for K = 0.
+// Scratch of one step inside the workspace.
+struct StepScratch {
+  float* partials;    // one per prologue item
+  float* mat_scale;   // one per matrix
+  int32_t* counters;  // [tickets: n_mats][done: n_mats * K * 3], zeroed per step
+  size_t counter_bytes;
+  int n_mats;
+};
+
 void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
-                  const float* ns_coeffs, int32_t ns_steps, float* partials,
-                  int32_t* done, int done_count, int fault, bool fresh,
-                  cudaStream_t st, Recorder* rec) {
+                  const float* ns_coeffs, int32_t ns_steps, const StepScratch& sc,
+                  int fault, bool fresh, cudaStream_t st, Recorder* rec) {
   HyperDev hd{h.momentum, h.lr, h.weight_decay, h.eps_row, h.eps_frob,
               h.nesterov, h.eq_r};
+  int32_t* tickets = sc.counters;
+  int32_t* done = sc.counters + sc.n_mats;
+  cudaMemsetAsync(sc.counters, 0, sc.counter_bytes, st);
   muon_prologue_kernel<<<static_cast<unsigned>(t.n_items), kProThreads,
-                         t.pro_smem, st>>>(t.mats, t.items, hd, partials);
+                         t.pro_smem, st>>>(t.mats, t.items, hd, sc.partials, tickets,
+                                           sc.mat_scale);
   if (rec) rec->after(MUON_KIND_PROLOGUE);
 
   if (ns_steps == 0) {
     muon_final_noiter_kernel<<<static_cast<unsigned>(t.n_items), kProThreads, 0,
-                               st>>>(t.mats, t.items, partials, h.lr,
-                                     h.weight_decay, h.eps_frob);
+                               st>>>(t.mats, t.items, sc.mat_scale, h.lr,
+                                     h.weight_decay);
     if (rec) rec->after(MUON_KIND_FINAL);
   }
   if (ns_steps > 0) {
@@ -346,7 +365,7 @@ void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
     p.gram = t.gram;
     p.poly = t.poly;
     p.apply = t.apply;
-    p.partials = partials;
+    p.mat_scale = sc.mat_scale;
     p.err = t.err;
     p.done = done;
     p.n_gram = t.n_gram;
@@ -363,7 +382,6 @@ void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
     p.lr = h.lr;
     p.wd = h.weight_decay;
     p.eps_frob = h.eps_frob;
-    cudaMemsetAsync(done, 0, static_cast<size_t>(done_count) * sizeof(int32_t), st);
     const long long items =
         static_cast<long long>(ns_steps) * (t.n_gram + t.n_poly + t.n_apply);
     const int clusters =
@@ -495,9 +513,12 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
   sort_tiles(plan->apply);
   plan->part_off = off;
   off = align_up(off + plan->items.size() * sizeof(float), 1024);
-  plan->done_off = off;
-  off = align_up(off + static_cast<size_t>(n_mats) * std::max(max_ns_steps, 1) * 3 *
-                           sizeof(int32_t), 1024);
+  plan->scale_off = off;
+  off = align_up(off + static_cast<size_t>(n_mats) * sizeof(float), 1024);
+  plan->counter_off = off;
+  plan->counter_bytes = static_cast<size_t>(n_mats) * (1 + 3 * std::max(max_ns_steps, 1)) *
+                        sizeof(int32_t);
+  off = align_up(off + plan->counter_bytes, 1024);
   plan->ws_bytes = off;
 
   // Device table.
@@ -676,11 +697,13 @@ muon_status_t muon_step_batched(muon_plan_t* plan, const muon_matrix_t* mats,
                  plan->d_poly, static_cast<int>(plan->poly.size()),
                  plan->d_apply, static_cast<int>(plan->apply.size()),
                  plan->d_err, plan->num_sms, plan->pro_smem, plan->max_clusters};
-  float* partials = reinterpret_cast<float*>(ws + plan->part_off);
-  int32_t* done = reinterpret_cast<int32_t*>(ws + plan->done_off);
+  StepScratch sc{reinterpret_cast<float*>(ws + plan->part_off),
+                 reinterpret_cast<float*>(ws + plan->scale_off),
+                 reinterpret_cast<int32_t*>(ws + plan->counter_off),
+                 plan->counter_bytes, plan->n_mats};
   Recorder rec(plan, st);
-  enqueue_step(t, *hyper, ns_coeffs, ns_steps, partials, done, plan->n_mats * ns_steps * 3,
-               plan->fault, changed, st, plan->timing ? &rec : nullptr);
+  enqueue_step(t, *hyper, ns_coeffs, ns_steps, sc, plan->fault, changed, st,
+               plan->timing ? &rec : nullptr);
   rec.finish();
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
@@ -859,9 +882,12 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
   sort_tiles_by_k(g_na_apply, n_apply);
   const size_t part_off = off;
   off = align_up(off + static_cast<size_t>(n_items) * sizeof(float), 1024);
-  const size_t done_off = off;
-  off = align_up(off + static_cast<size_t>(n_mats) * std::max(ns_steps, 1) * 3 *
-                           sizeof(int32_t), 1024);
+  const size_t scale_off = off;
+  off = align_up(off + static_cast<size_t>(n_mats) * sizeof(float), 1024);
+  const size_t counter_off = off;
+  const size_t counter_bytes =
+      static_cast<size_t>(n_mats) * (1 + 3 * std::max(ns_steps, 1)) * sizeof(int32_t);
+  off = align_up(off + counter_bytes, 1024);
   const size_t ws_bytes = off;
 
   // Layout of the device array: [error word][tables][workspace].
@@ -940,10 +966,10 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
                  reinterpret_cast<const NsTile*>(base + apply_off), n_apply,
                  reinterpret_cast<int32_t*>(base), num_sms, pro_smem,
                  g_noalloc_clusters[dev]};
-  float* partials = reinterpret_cast<float*>(ws + part_off);
-  int32_t* done = reinterpret_cast<int32_t*>(ws + done_off);
-  enqueue_step(t, *hyper, ns_coeffs, ns_steps, partials, done, n_mats * ns_steps * 3, 0,
-               true, st, nullptr);
+  StepScratch sc{reinterpret_cast<float*>(ws + part_off),
+                 reinterpret_cast<float*>(ws + scale_off),
+                 reinterpret_cast<int32_t*>(ws + counter_off), counter_bytes, n_mats};
+  enqueue_step(t, *hyper, ns_coeffs, ns_steps, sc, 0, true, st, nullptr);
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
 }

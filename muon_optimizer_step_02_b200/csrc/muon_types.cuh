@@ -9,10 +9,10 @@ namespace muonb200 {
 
 constexpr int kTileM = 128;       // rows of a tile held by one CTA (TMEM lanes)
 constexpr int kTileK = 64;        // K per pipeline stage (one 128-B swizzle row)
+constexpr int kPairTile = 256;    // CTA-pair tile: 256 rows (128 per CTA) x 256 cols
 constexpr int kProRows = 32;      // rows per prologue work item
 constexpr int kProThreads = 256;  // 8 warps
-constexpr int kProCachedChunks = 8;  // row chunks (of 256 elements) kept in
-                                     // registers: rows up to 2048 are read once
+constexpr int kProBatch = 2;      // row chunks (of 256 elements) in flight per warp
 
 // Per-matrix record.  Tensor maps first (64-byte aligned), pointers after.
 struct alignas(64) MatDev {
@@ -20,6 +20,9 @@ struct alignas(64) MatDev {
   CUtensorMap tm_xn[2];  // X ping/pong as an MN-major operand, box 64 x 64
   CUtensorMap tm_a;      // A = X X^T (m x m), box 64 x 128
   CUtensorMap tm_b;      // B = b A + c A A (m x m), box 64 x 128
+  CUtensorMap tm_xs[2];  // X ping/pong for 32 x 32 epilogue stores
+  CUtensorMap tm_as;     // A for 32 x 32 epilogue stores
+  CUtensorMap tm_bs;     // B for 32 x 32 epilogue stores
   __nv_bfloat16* x[2];   // m x ldx each
   __nv_bfloat16* a;      // m x lda
   __nv_bfloat16* b;      // m x lda

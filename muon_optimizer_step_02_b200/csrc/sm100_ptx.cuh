@@ -328,3 +328,39 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) 
 }
 
 }  // namespace muonb200
+
+// ---------------------------------------------------------------- TMA stores
+namespace muonb200 {
+
+// 2-D tiled bulk tensor store shared -> global (elements outside the tensor
+// are not written).  x is the innermost coordinate; x * elem_size % 16 == 0.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, uint32_t src,
+                                             int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(tm)),
+      "r"(src), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until the committed bulk stores of this thread have read their
+// shared-memory source (the buffer may be rewritten).
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Wait until the committed bulk stores of this thread are complete.
+__device__ __forceinline__ void bulk_wait_group0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Makes this thread's shared-memory writes visible to the async proxy (TMA).
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+}  // namespace muonb200

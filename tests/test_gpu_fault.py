@@ -1,0 +1,37 @@
+"""Failure detection without a GPU fault: the test hook makes the first
+stage of the first tile never arrive, so the tensor-core kernel's bounded
+wait runs out (about one second), the kernel records the error word, drains
+its own copies and MMAs, frees TMEM and returns.  The host must read
+MUON_ERR_TIMEOUT, and the same plan must work normally afterwards."""
+import numpy as np
+import pytest
+
+from gpu_harness import GpuMuon, check_step
+from muon_optimizer_step_02_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+def test_bounded_wait_timeout_is_reported_and_recoverable():
+    import time
+
+    import torch
+    from muon_optimizer_step_02_b200 import binding as B
+    h = wl.Hyper(momentum=0.95, lr=0.02, weight_decay=0.1)
+    w = wl.custom([(256, 512), (512, 256)], h, [wl.FIXED_QUINTIC] * 5,
+                  wid=500)
+    g = GpuMuon(w)
+    g.plan.set_fault(1)
+    t0 = time.time()
+    g.step(g.grads(0))
+    status = g.plan.last_error()          # synchronises the stream
+    elapsed = time.time() - t0
+    assert status == B.MUON_ERR_TIMEOUT
+    assert elapsed < 30.0
+    # the error word is cleared by the read
+    assert g.plan.last_error() == B.MUON_OK
+    # the context and the plan still work: a clean step matches the oracle
+    g.plan.set_fault(0)
+    torch.cuda.synchronize()
+    g2 = GpuMuon(w)
+    check_step(g2, 0, [0, 1])
