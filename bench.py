@@ -40,6 +40,39 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
                   "bf16_tflops_sustained": 1400.0}
 
 
+def kernel_source_hash() -> str:
+    """sha256 over the CUDA sources, to tell whether a recorded ncu traffic
+    figure still belongs to the kernels being timed."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    pat = os.path.join(ROOT, "muon_optimizer_step_02_b200", "csrc", "*")
+    for f in sorted(glob.glob(pat)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(os.path.basename(f).encode())
+            with open(f, "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel: str, workload: int):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary
+    (profiles/roofline_traffic.json), or None if it was taken on other
+    kernel sources or another workload."""
+    path = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+    try:
+        with open(path) as f:
+            doc = json.load(f)
+    except (OSError, ValueError):
+        return None
+    rec = doc.get(kernel)
+    if not rec or rec.get("workload") != workload:
+        return None
+    if rec.get("source_sha256") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -279,12 +312,16 @@ def run_ours(args, rank, world, local_rank):
     if dom in ns_kinds:
         per_launch = flops[dom]
         achieved = per_launch / (ms_dom / launches_dom / 1e3) / 1e12
-        roof = {"kernel": f"ns_mega_pair_kernel (all {len(w.coeffs)} "
-                          "Newton-Schulz steps)" if dom == "ns" else dom,
+        kname = "ns_mega_pair_kernel" if dom == "ns" else dom
+        roof = {"kernel": f"{kname} (all {len(w.coeffs)} Newton-Schulz steps)"
+                if dom == "ns" else dom,
                 "bound": "tensor",
                 "achieved": round(achieved, 2), "peak": sustained,
                 "unit": "TFLOP/s", "frac": round(achieved / sustained, 4),
-                "traffic": None, "peak_source": f"{peak_src} sustained bf16"}
+                "traffic": recorded_traffic(kname, args.workload),
+                "traffic_unit": "bytes per launch (ncu dram read + write)",
+                "flops_per_launch": per_launch,
+                "peak_source": f"{peak_src} sustained bf16"}
     else:
         per_launch = rep.state_bytes()["prologue"]
         achieved = per_launch / (ms_dom / launches_dom / 1e3) / 1e9

@@ -1,10 +1,10 @@
 // All K Newton-Schulz steps of every matrix in one persistent launch on CTA
 // pairs (tcgen05.mma.cta_group::2, 256 x 256 tiles).
 //
-// The work list is, for k = 0..K-1: the gram tiles of every matrix, then the
-// poly tiles, then the apply tiles.  Cluster c takes items c, c + C, c + 2C,
-// ... in that order.  An item waits (in its producer, before loading) until
-// the phase it reads is complete for its matrix:
+// The work list (built on the host by schedule.h) holds the gram, poly and
+// apply pair tiles of every step of every matrix.  Cluster c takes items c,
+// c + C, c + 2C, ... in that order.  An item waits (in its producer, before
+// loading) until the phase it reads is complete for its matrix:
 //   gram(k)  reads X_k   <- every apply(k-1) tile of the matrix (k > 0)
 //   poly(k)  reads A     <- every gram(k) tile of the matrix
 //   apply(k) reads B', X <- every poly(k) tile of the matrix
@@ -53,13 +53,11 @@ constexpr int kMegaStages = 6;
 
 struct MegaParams {
   const MatDev* mats;
-  const NsTile* gram;     // pair tiles, K = n
-  const NsTile* poly;     // pair tiles, K = m
-  const NsTile* apply;    // pair tiles, K = m
+  const SchedItem* items; // the schedule (host-built list, see schedule.h)
   const float* mat_scale; // per-matrix Frobenius scale from the prologue
   int32_t* err;
   int32_t* done;          // [mat][step][phase] completion counts, zeroed
-  int32_t n_gram, n_poly, n_apply;
+  int32_t n_items;
   int32_t steps;
   int32_t fault, fresh;
   float a[kMegaMaxSteps], b[kMegaMaxSteps], c[kMegaMaxSteps];
@@ -110,20 +108,14 @@ struct MegaItem {
 };
 
 __device__ __forceinline__ MegaItem mega_item(const MegaParams& p, int g) {
-  const int per_step = p.n_gram + p.n_poly + p.n_apply;
+  const SchedItem si = p.items[g];
   MegaItem it;
-  it.k = g / per_step;
-  int r = g - it.k * per_step;
-  if (r < p.n_gram) {
-    it.mode = kModeGram;
-    it.tl = p.gram[r];
-  } else if (r < p.n_gram + p.n_poly) {
-    it.mode = kModePoly;
-    it.tl = p.poly[r - p.n_gram];
-  } else {
-    it.mode = kModeApply;
-    it.tl = p.apply[r - p.n_gram - p.n_poly];
-  }
+  it.tl.mat = si.mat;
+  it.tl.ti = si.ti;
+  it.tl.tj = si.tj;
+  it.tl.kt = si.kt;
+  it.mode = si.mode;
+  it.k = si.k;
   return it;
 }
 
@@ -178,7 +170,7 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
-  const int total = p.steps * (p.n_gram + p.n_poly + p.n_apply);
+  const int total = p.n_items;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {

@@ -1,11 +1,13 @@
 // C ABI of the batched Muon step and the batched EMA (include/muon_b200.h):
-// argument validation, the plan (shapes -> workspace layout, work lists and
-// tile lists, built once), TMA descriptor encoding, and the launch sequence
+// argument validation, the plan (shapes -> workspace layout, prologue work
+// items and the Newton-Schulz schedule, built once), TMA descriptor
+// encoding, and the launch sequence on the caller's stream:
 //
-//   prologue  ->  K x (gram -> poly -> apply)      (1 + 3K launches)
+//   counter reset (memset) -> prologue -> all Newton-Schulz steps (one
+//   persistent CTA-pair kernel)                      or, with 0 steps,
+//   counter reset -> prologue -> finisher
 //
-// on the caller's stream.  No device memory is allocated after
-// muon_plan_create.
+// No device memory is allocated after muon_plan_create.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -23,6 +25,7 @@
 #include "k_ns_mega.cuh"
 #include "k_prologue.cuh"
 #include "muon_types.cuh"
+#include "schedule.h"
 
 using namespace muonb200;
 
@@ -30,9 +33,9 @@ namespace {
 
 constexpr int kMaxNsSteps = 16;
 constexpr int kMaxMats = 4096;
-constexpr int kMaxLaunchesPerStep = 1 + 3 * kMaxNsSteps;
+constexpr int kMaxLaunchesPerStep = 2;
 constexpr int kTimingSlots = 64;
-constexpr size_t kProSmemCap = 48 * 1024;   // four prologue blocks per SM
+constexpr size_t kProSmemCap = 48 * 1024;   // staging of the transposed write
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -79,12 +82,56 @@ bool encode_bf16_2d(CUtensorMap* tm, void* base, int rows, int cols, int ld,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Per-matrix geometry and its place in the workspace.
 struct Geom {
   int rows, cols, m, n, ldx, lda, transposed;
   size_t x_off[2], a_off, b_off;
   int part_first, part_count;
-  int n_sym_tiles, n_apply_tiles;
+  int t2, tn;                      // 256-blocks of m and of n
+  int n_sym_tiles, n_apply_tiles;  // pair tiles per phase
 };
+
+int pro_rows_per_item(int rows, int cols) {
+  if (rows <= cols) return kProRows;
+  size_t per_row = static_cast<size_t>(cols + 2) * 2;
+  int rt = static_cast<int>(std::min<size_t>(kProRows, kProSmemCap / per_row));
+  if (rt >= 8) rt &= ~7;
+  return std::max(rt, 1);
+}
+
+// Shape checks, geometry, and the workspace offsets of X ping/pong, A, B'.
+muon_status_t layout_matrix(int rows, int cols, Geom& g, size_t& off) {
+  if (rows < 1 || cols < 1) return MUON_ERR_INVALID_ARG;
+  // tile coordinates are 16-bit; keep every dimension well inside
+  if (rows > (1 << 20) || cols > (1 << 20) ||
+      static_cast<long long>(rows) * cols > (1ll << 31) - 1)
+    return MUON_ERR_UNSUPPORTED;
+  g.rows = rows;
+  g.cols = cols;
+  g.transposed = rows > cols;
+  g.m = std::min(rows, cols);
+  g.n = std::max(rows, cols);
+  g.ldx = static_cast<int>(align_up(g.n, 8));
+  g.lda = static_cast<int>(align_up(g.m, 8));
+  for (int b = 0; b < 2; ++b) {
+    g.x_off[b] = off;
+    off = align_up(off + static_cast<size_t>(g.m) * g.ldx * 2, 1024);
+  }
+  g.a_off = off;
+  off = align_up(off + static_cast<size_t>(g.m) * g.lda * 2, 1024);
+  g.b_off = off;
+  off = align_up(off + static_cast<size_t>(g.m) * g.lda * 2, 1024);
+  g.t2 = ceil_div(g.m, kPairTile);
+  g.tn = ceil_div(g.n, kPairTile);
+  g.n_sym_tiles = g.t2 * (g.t2 + 1) / 2;
+  g.n_apply_tiles = g.t2 * g.tn;
+  return MUON_OK;
+}
+
+size_t counter_bytes_for(int n_mats, int steps) {
+  // one prologue ticket per matrix + one count per (matrix, step, phase)
+  return static_cast<size_t>(n_mats) * (1 + 3 * std::max(steps, 1)) * sizeof(int32_t);
+}
 
 struct TimingSlot {
   cudaEvent_t ev[kMaxLaunchesPerStep + 1];
@@ -105,7 +152,6 @@ struct muon_plan {
   int max_ns = 0;
   std::vector<Geom> geom;
   std::vector<ProItem> items;
-  std::vector<NsTile> gram, poly, apply;
   size_t ws_bytes = 0;
   size_t part_off = 0;
   size_t scale_off = 0;
@@ -114,13 +160,22 @@ struct muon_plan {
   size_t pro_smem = 0;
   int max_clusters = 0;
 
-  // device table: [MatDev x n_mats][ProItem][gram][poly][apply][err]
+  // Newton-Schulz schedule for `sched_steps` steps (rebuilt when the step
+  // count of a call changes)
+  std::vector<SchedMatrix> smats;
+  std::vector<SchedItem> sched;
+  std::vector<SchedGroup> sgroups;
+  std::vector<int> sorder;
+  std::vector<double> scl;
+  int sched_steps = -1;
+  long long sched_len = 0;
+  long long sched_cap = 0;
+
+  // device table: [MatDev x n_mats][ProItem][SchedItem x cap][err]
   void* d_block = nullptr;
   MatDev* d_mats = nullptr;
   ProItem* d_items = nullptr;
-  NsTile* d_gram = nullptr;
-  NsTile* d_poly = nullptr;
-  NsTile* d_apply = nullptr;
+  SchedItem* d_sched = nullptr;
   int32_t* d_err = nullptr;
 
   std::vector<MatDev> h_mats;     // what the device table holds now
@@ -150,6 +205,7 @@ void harvest(muon_plan* plan, TimingSlot& s) {
   s.pending = false;
 }
 
+// CUDA events on the launching stream around each launch of one call.
 struct Recorder {
   muon_plan* plan;
   cudaStream_t stream;
@@ -173,34 +229,25 @@ struct Recorder {
   }
 };
 
-int pro_rows_per_item(int rows, int cols) {
-  if (rows <= cols) return kProRows;
-  size_t per_row = static_cast<size_t>(cols + 2) * 2;
-  int rt = static_cast<int>(std::min<size_t>(kProRows, kProSmemCap / per_row));
-  if (rt >= 8) rt &= ~7;
-  return std::max(rt, 1);
-}
-
-void sort_tiles(std::vector<NsTile>& v) {
-  std::stable_sort(v.begin(), v.end(),
-                   [](const NsTile& a, const NsTile& b) { return a.kt > b.kt; });
-}
-
 // Everything the launch sequence needs: where the device tables are.
 struct LaunchTables {
   const MatDev* mats;
   const ProItem* items;
   int n_items;
-  const NsTile* gram;
-  int n_gram;
-  const NsTile* poly;
-  int n_poly;
-  const NsTile* apply;
-  int n_apply;
+  const SchedItem* sched;
+  long long n_sched;
   int32_t* err;
-  int num_sms;
   size_t pro_smem;
-  int max_clusters;   // co-resident clusters of the Newton-Schulz kernel
+  int clusters;       // clusters the schedule was built for (all resident)
+};
+
+// Scratch of one step inside the workspace.
+struct StepScratch {
+  float* partials;    // one per prologue item
+  float* mat_scale;   // one per matrix
+  int32_t* counters;  // [tickets: n_mats][done: n_mats * K * 3], zeroed per step
+  size_t counter_bytes;
+  int n_mats;
 };
 
 muon_status_t validate_hyper(const muon_hyper_t* hyper, const float* ns_coeffs,
@@ -275,24 +322,44 @@ bool fill_caller_fields(MatDev& d, const muon_matrix_t& mt) {
   return true;
 }
 
-// Clusters of two that can be resident at once (the persistent schedule
-// relies on every launched cluster being resident); 0 on failure.
-int query_max_clusters() {
+bool set_kernel_attributes(size_t pro_smem) {
   if (cudaFuncSetAttribute(ns_mega_pair_kernel,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kMegaSmemBytes)) != cudaSuccess)
-    return 0;
+    return false;
+  if (pro_smem > 48 * 1024 &&
+      cudaFuncSetAttribute(muon_prologue_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(pro_smem)) != cudaSuccess)
+    return false;
+  return true;
+}
+
+cudaLaunchConfig_t pair_launch_config(int clusters, cudaStream_t st,
+                                      cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2);
+  cfg.gridDim = dim3(2 * clusters);
   cfg.blockDim = dim3(kNsThreads);
   cfg.dynamicSmemBytes = kMegaSmemBytes;
-  cudaLaunchAttribute attr[1];
+  cfg.stream = st;
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  return cfg;
+}
+
+// Clusters of two that can be resident at once (the persistent schedule
+// relies on every launched cluster being resident); 0 on failure.
+int query_max_clusters() {
+  if (!set_kernel_attributes(0)) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pair_launch_config(1, nullptr, attr);
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, ns_mega_pair_kernel, &cfg) != cudaSuccess) {
     cudaGetLastError();
@@ -301,45 +368,14 @@ int query_max_clusters() {
   return n;
 }
 
-
-// Pair tiles of one matrix: symmetric products over upper 256 x 256 blocks,
-// the apply over all 256 x 256 blocks of X.  Returns false on overflow.
-bool append_pair_tiles(int mat, const Geom& g, NsTile* gram, NsTile* poly,
-                       int& n_gram, int cap_gram, NsTile* apply, int& n_apply,
-                       int cap_apply) {
-  const int t2 = ceil_div(g.m, kPairTile);
-  for (int ti = 0; ti < t2; ++ti)
-    for (int tj = ti; tj < t2; ++tj) {
-      if (n_gram >= cap_gram) return false;
-      gram[n_gram] = NsTile{static_cast<uint16_t>(mat), static_cast<uint16_t>(ti),
-                            static_cast<uint16_t>(tj),
-                            static_cast<uint16_t>(ceil_div(g.n, kTileK))};
-      poly[n_gram] = NsTile{static_cast<uint16_t>(mat), static_cast<uint16_t>(ti),
-                            static_cast<uint16_t>(tj),
-                            static_cast<uint16_t>(ceil_div(g.m, kTileK))};
-      ++n_gram;
-    }
-  const int tn = ceil_div(g.n, kPairTile);
-  for (int ti = 0; ti < t2; ++ti)
-    for (int tj = 0; tj < tn; ++tj) {
-      if (n_apply >= cap_apply) return false;
-      apply[n_apply++] = NsTile{static_cast<uint16_t>(mat), static_cast<uint16_t>(ti),
-                                static_cast<uint16_t>(tj),
-                                static_cast<uint16_t>(ceil_div(g.m, kTileK))};
-    }
-  return true;
+void fill_sched_matrix(SchedMatrix& s, const Geom& g) {
+  s.m = g.m;
+  s.n = g.n;
+  s.t2 = g.t2;
+  s.tn = g.tn;
 }
 
-// prologue -> K x (gram -> poly -> apply), or prologue -> final for K = 0.
-// Scratch of one step inside the workspace.
-struct StepScratch {
-  float* partials;    // one per prologue item
-  float* mat_scale;   // one per matrix
-  int32_t* counters;  // [tickets: n_mats][done: n_mats * K * 3], zeroed per step
-  size_t counter_bytes;
-  int n_mats;
-};
-
+// counter reset -> prologue -> Newton-Schulz (or finisher for 0 steps).
 void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
                   const float* ns_coeffs, int32_t ns_steps, const StepScratch& sc,
                   int fault, bool fresh, cudaStream_t st, Recorder* rec) {
@@ -358,49 +394,30 @@ void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
                                st>>>(t.mats, t.items, sc.mat_scale, h.lr,
                                      h.weight_decay);
     if (rec) rec->after(MUON_KIND_FINAL);
+    return;
   }
-  if (ns_steps > 0) {
-    MegaParams p{};
-    p.mats = t.mats;
-    p.gram = t.gram;
-    p.poly = t.poly;
-    p.apply = t.apply;
-    p.mat_scale = sc.mat_scale;
-    p.err = t.err;
-    p.done = done;
-    p.n_gram = t.n_gram;
-    p.n_poly = t.n_poly;
-    p.n_apply = t.n_apply;
-    p.steps = ns_steps;
-    p.fault = fault;
-    p.fresh = fresh ? 1 : 0;
-    for (int k = 0; k < ns_steps; ++k) {
-      p.a[k] = ns_coeffs[3 * k + 0];
-      p.b[k] = ns_coeffs[3 * k + 1];
-      p.c[k] = ns_coeffs[3 * k + 2];
-    }
-    p.lr = h.lr;
-    p.wd = h.weight_decay;
-    p.eps_frob = h.eps_frob;
-    const long long items =
-        static_cast<long long>(ns_steps) * (t.n_gram + t.n_poly + t.n_apply);
-    const int clusters =
-        static_cast<int>(std::max<long long>(1, std::min<long long>(t.max_clusters, items)));
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * clusters);
-    cfg.blockDim = dim3(kNsThreads);
-    cfg.dynamicSmemBytes = kMegaSmemBytes;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, ns_mega_pair_kernel, p);
-    if (rec) rec->after(MUON_KIND_NS);
+  MegaParams p{};
+  p.mats = t.mats;
+  p.items = t.sched;
+  p.mat_scale = sc.mat_scale;
+  p.err = t.err;
+  p.done = done;
+  p.n_items = static_cast<int32_t>(t.n_sched);
+  p.steps = ns_steps;
+  p.fault = fault;
+  p.fresh = fresh ? 1 : 0;
+  for (int k = 0; k < ns_steps; ++k) {
+    p.a[k] = ns_coeffs[3 * k + 0];
+    p.b[k] = ns_coeffs[3 * k + 1];
+    p.c[k] = ns_coeffs[3 * k + 2];
   }
+  p.lr = h.lr;
+  p.wd = h.weight_decay;
+  p.eps_frob = h.eps_frob;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pair_launch_config(t.clusters, st, attr);
+  cudaLaunchKernelEx(&cfg, ns_mega_pair_kernel, p);
+  if (rec) rec->after(MUON_KIND_NS);
 }
 
 }  // namespace
@@ -423,7 +440,7 @@ const char* muon_status_string(muon_status_t s) {
 }
 
 int32_t muon_step_launches(int32_t ns_steps) {
-  // prologue, then one Newton-Schulz launch for all steps (or the K = 0
+  // prologue, then one Newton-Schulz launch for all steps (or the 0-step
   // finisher); the counter reset is a memset, not a kernel
   return ns_steps < 0 ? 0 : 2;
 }
@@ -440,86 +457,58 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
   if (!rows || !cols || n_mats < 1 || n_mats > kMaxMats) return MUON_ERR_INVALID_ARG;
   if (max_ns_steps < 0 || max_ns_steps > kMaxNsSteps) return MUON_ERR_UNSUPPORTED;
   for (int i = 0; i < n_mats; ++i) {
-    if (rows[i] < 1 || cols[i] < 1) return MUON_ERR_INVALID_ARG;
-    // tile coordinates are 16-bit; keep every dimension well inside
-    if (rows[i] > (1 << 20) || cols[i] > (1 << 20)) return MUON_ERR_UNSUPPORTED;
-    if (static_cast<long long>(rows[i]) * cols[i] > (1ll << 31) - 1)
-      return MUON_ERR_UNSUPPORTED;
+    Geom g;
+    size_t scratch = 0;
+    const muon_status_t vs = layout_matrix(rows[i], cols[i], g, scratch);
+    if (vs != MUON_OK) return vs;
   }
 
   muon_plan* plan = new (std::nothrow) muon_plan();
   if (!plan) return MUON_ERR_INVALID_ARG;
   plan->n_mats = n_mats;
   plan->max_ns = max_ns_steps;
-  if (cudaGetDevice(&plan->device) != cudaSuccess ||
-      cudaDeviceGetAttribute(&plan->num_sms, cudaDevAttrMultiProcessorCount,
-                             plan->device) != cudaSuccess) {
-    delete plan;
-    return MUON_ERR_CUDA;
-  }
 
-  // Geometry, workspace layout, prologue work items, tile lists.
+  // Geometry, workspace layout, prologue work items.
   size_t off = 0;
+  long long per_step_items = 0;
   plan->geom.resize(n_mats);
+  plan->smats.resize(n_mats);
   for (int i = 0; i < n_mats; ++i) {
     Geom& g = plan->geom[i];
-    g.rows = rows[i];
-    g.cols = cols[i];
-    g.transposed = rows[i] > cols[i];
-    g.m = std::min(rows[i], cols[i]);
-    g.n = std::max(rows[i], cols[i]);
-    g.ldx = static_cast<int>(align_up(g.n, 8));
-    g.lda = static_cast<int>(align_up(g.m, 8));
-    for (int b = 0; b < 2; ++b) {
-      g.x_off[b] = off;
-      off = align_up(off + static_cast<size_t>(g.m) * g.ldx * 2, 1024);
-    }
-    g.a_off = off;
-    off = align_up(off + static_cast<size_t>(g.m) * g.lda * 2, 1024);
-    g.b_off = off;
-    off = align_up(off + static_cast<size_t>(g.m) * g.lda * 2, 1024);
-
+    layout_matrix(rows[i], cols[i], g, off);
     const int rt = pro_rows_per_item(g.rows, g.cols);
     g.part_first = static_cast<int>(plan->items.size());
-    for (int r0 = 0; r0 < g.rows; r0 += rt) {
-      ProItem it{i, r0, std::min(rt, g.rows - r0), 0};
-      plan->items.push_back(it);
-    }
+    for (int r0 = 0; r0 < g.rows; r0 += rt)
+      plan->items.push_back(ProItem{i, r0, std::min(rt, g.rows - r0), 0});
     g.part_count = static_cast<int>(plan->items.size()) - g.part_first;
     if (g.transposed)
       plan->pro_smem = std::max(plan->pro_smem,
                                 static_cast<size_t>(rt) * (g.cols + 2) * 2);
-
-    {
-      const int t2 = ceil_div(g.m, kPairTile), tn = ceil_div(g.n, kPairTile);
-      const size_t ng = plan->gram.size(), na = plan->apply.size();
-      plan->gram.resize(ng + t2 * (t2 + 1) / 2);
-      plan->poly.resize(ng + t2 * (t2 + 1) / 2);
-      plan->apply.resize(na + static_cast<size_t>(t2) * tn);
-      int n_gram = 0, n_apply = 0;
-      append_pair_tiles(i, g, plan->gram.data() + ng, plan->poly.data() + ng, n_gram,
-                        t2 * (t2 + 1) / 2, plan->apply.data() + na, n_apply, t2 * tn);
-      g.n_sym_tiles = n_gram;
-      g.n_apply_tiles = n_apply;
-    }
+    fill_sched_matrix(plan->smats[i], g);
+    per_step_items += 2 * g.n_sym_tiles + g.n_apply_tiles;
   }
-  if (plan->items.size() > 0x7FFFFFFF ||
-      plan->gram.size() > 0x7FFFFFFF || plan->apply.size() > 0x7FFFFFFF) {
+  plan->sched_cap = per_step_items * std::max(max_ns_steps, 1);
+  if (plan->items.size() > 0x7FFFFFFF || plan->sched_cap > 0x7FFFFFFF) {
     delete plan;
     return MUON_ERR_UNSUPPORTED;
   }
-  sort_tiles(plan->gram);
-  sort_tiles(plan->poly);
-  sort_tiles(plan->apply);
   plan->part_off = off;
   off = align_up(off + plan->items.size() * sizeof(float), 1024);
   plan->scale_off = off;
   off = align_up(off + static_cast<size_t>(n_mats) * sizeof(float), 1024);
   plan->counter_off = off;
-  plan->counter_bytes = static_cast<size_t>(n_mats) * (1 + 3 * std::max(max_ns_steps, 1)) *
-                        sizeof(int32_t);
+  plan->counter_bytes = counter_bytes_for(n_mats, max_ns_steps);
   off = align_up(off + plan->counter_bytes, 1024);
   plan->ws_bytes = off;
+
+  if (cudaGetDevice(&plan->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&plan->num_sms, cudaDevAttrMultiProcessorCount,
+                             plan->device) != cudaSuccess) {
+    cudaGetLastError();
+    delete plan;
+    return MUON_ERR_CUDA;
+  }
+  plan->max_clusters = query_max_clusters();
 
   // Device table.
   size_t t_off = 0;
@@ -527,15 +516,12 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
   t_off = align_up(t_off + sizeof(MatDev) * n_mats, 256);
   const size_t items_off = t_off;
   t_off = align_up(t_off + sizeof(ProItem) * plan->items.size(), 256);
-  const size_t gram_off = t_off;
-  t_off = align_up(t_off + sizeof(NsTile) * plan->gram.size(), 256);
-  const size_t poly_off = t_off;
-  t_off = align_up(t_off + sizeof(NsTile) * plan->poly.size(), 256);
-  const size_t apply_off = t_off;
-  t_off = align_up(t_off + sizeof(NsTile) * plan->apply.size(), 256);
+  const size_t sched_off = t_off;
+  t_off = align_up(t_off + sizeof(SchedItem) * plan->sched_cap, 256);
   const size_t err_off = t_off;
   t_off += 256;
-  if (cudaMalloc(&plan->d_block, t_off) != cudaSuccess) {
+  if (plan->max_clusters <= 0 || !set_kernel_attributes(plan->pro_smem) ||
+      cudaMalloc(&plan->d_block, t_off) != cudaSuccess) {
     cudaGetLastError();
     delete plan;
     return MUON_ERR_CUDA;
@@ -543,26 +529,12 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
   char* base = static_cast<char*>(plan->d_block);
   plan->d_mats = reinterpret_cast<MatDev*>(base + mats_off);
   plan->d_items = reinterpret_cast<ProItem*>(base + items_off);
-  plan->d_gram = reinterpret_cast<NsTile*>(base + gram_off);
-  plan->d_poly = reinterpret_cast<NsTile*>(base + poly_off);
-  plan->d_apply = reinterpret_cast<NsTile*>(base + apply_off);
+  plan->d_sched = reinterpret_cast<SchedItem*>(base + sched_off);
   plan->d_err = reinterpret_cast<int32_t*>(base + err_off);
-  bool ok =
+  const bool ok =
       cudaMemcpy(plan->d_items, plan->items.data(), sizeof(ProItem) * plan->items.size(),
                  cudaMemcpyHostToDevice) == cudaSuccess &&
-      cudaMemcpy(plan->d_gram, plan->gram.data(), sizeof(NsTile) * plan->gram.size(),
-                 cudaMemcpyHostToDevice) == cudaSuccess &&
-      cudaMemcpy(plan->d_poly, plan->poly.data(), sizeof(NsTile) * plan->poly.size(),
-                 cudaMemcpyHostToDevice) == cudaSuccess &&
-      cudaMemcpy(plan->d_apply, plan->apply.data(), sizeof(NsTile) * plan->apply.size(),
-                 cudaMemcpyHostToDevice) == cudaSuccess &&
       cudaMemset(plan->d_err, 0, sizeof(int32_t)) == cudaSuccess;
-  ok = ok &&
-       (plan->max_clusters = query_max_clusters()) > 0 &&
-       cudaFuncSetAttribute(muon_prologue_kernel,
-                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                            static_cast<int>(std::max<size_t>(plan->pro_smem, 1024))) ==
-           cudaSuccess;
   if (!ok) {
     cudaGetLastError();
     cudaFree(plan->d_block);
@@ -570,6 +542,10 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
     return MUON_ERR_CUDA;
   }
   plan->h_mats.resize(n_mats);
+  plan->sched.resize(plan->sched_cap);
+  plan->sgroups.resize(static_cast<size_t>(n_mats) * std::max(max_ns_steps, 1) * 3);
+  plan->sorder.resize(n_mats);
+  plan->scl.resize(plan->max_clusters);
   *out = plan;
   return MUON_OK;
 }
@@ -658,7 +634,7 @@ muon_status_t muon_step_batched(muon_plan_t* plan, const muon_matrix_t* mats,
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  // ---- per-matrix device table (uploaded only when something changed)
+  // ---- per-matrix device table and schedule (uploaded only on change)
   char* ws = static_cast<char*>(workspace);
   std::vector<MatDev>& hm = plan->h_mats;
   if (plan->enc_ws != workspace) {
@@ -674,12 +650,15 @@ muon_status_t muon_step_batched(muon_plan_t* plan, const muon_matrix_t* mats,
   bool changed = !plan->h_valid;
   for (int i = 0; i < plan->n_mats; ++i)
     changed |= fill_caller_fields(hm[i], mats[i]);
-  if (changed) {
+  const bool resched = ns_steps > 0 && ns_steps != plan->sched_steps;
+  if (changed || resched) {
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return MUON_ERR_CUDA;
     // A host-to-device table copy cannot be captured from pageable memory:
-    // run one call with the same buffers before capturing.
+    // run one call with the same buffers and step count before capturing.
     if (cap != cudaStreamCaptureStatusNone) return MUON_ERR_UNSUPPORTED;
+  }
+  if (changed) {
     // Pageable source: the call returns once the bytes are staged, so the
     // host table may change right after; the copy is ordered on `st` after
     // every earlier kernel of this plan.
@@ -690,17 +669,29 @@ muon_status_t muon_step_batched(muon_plan_t* plan, const muon_matrix_t* mats,
     }
     plan->h_valid = true;
   }
+  if (resched) {
+    const long long n = build_schedule(plan->smats.data(), plan->n_mats, ns_steps,
+                                       plan->max_clusters, plan->sched.data(),
+                                       plan->sched_cap, plan->sgroups.data(),
+                                       plan->sorder.data(), plan->scl.data());
+    if (n < 0) return MUON_ERR_UNSUPPORTED;
+    if (cudaMemcpyAsync(plan->d_sched, plan->sched.data(), sizeof(SchedItem) * n,
+                        cudaMemcpyHostToDevice, st) != cudaSuccess) {
+      plan->sched_steps = -1;
+      return MUON_ERR_CUDA;
+    }
+    plan->sched_steps = ns_steps;
+    plan->sched_len = n;
+  }
 
   // ---- launches
   LaunchTables t{plan->d_mats, plan->d_items, static_cast<int>(plan->items.size()),
-                 plan->d_gram, static_cast<int>(plan->gram.size()),
-                 plan->d_poly, static_cast<int>(plan->poly.size()),
-                 plan->d_apply, static_cast<int>(plan->apply.size()),
-                 plan->d_err, plan->num_sms, plan->pro_smem, plan->max_clusters};
+                 plan->d_sched, plan->sched_len, plan->d_err, plan->pro_smem,
+                 plan->max_clusters};
   StepScratch sc{reinterpret_cast<float*>(ws + plan->part_off),
                  reinterpret_cast<float*>(ws + plan->scale_off),
                  reinterpret_cast<int32_t*>(ws + plan->counter_off),
-                 plan->counter_bytes, plan->n_mats};
+                 counter_bytes_for(plan->n_mats, ns_steps), plan->n_mats};
   Recorder rec(plan, st);
   enqueue_step(t, *hyper, ns_coeffs, ns_steps, sc, plan->fault, changed, st,
                plan->timing ? &rec : nullptr);
@@ -763,14 +754,15 @@ muon_status_t ema_update_batched(float* const* ema, const float* const* params,
 // allocate device memory.
 //
 // All of the step's scratch (the per-matrix records with their TMA
-// descriptors, the work and tile lists, the error word, and the working
-// matrices X, A, B' and the norm partials) lives in one file-scope device
-// array, g_noalloc_scratch, of MUON_NOALLOC_SCRATCH_BYTES.  The CUDA runtime
-// reserves it on every device where this library's kernels are loaded, for
-// the life of the process.  Host code must not pass the array's name to a
-// kernel (in host code it names a host-side stand-in); the device address
-// comes from cudaGetSymbolAddress, looked up once per device with that
-// device current, on the first call made on that device.
+// descriptors, the work items and the schedule, the error word, and the
+// working matrices X, A, B', the norm partials and the counters) lives in one
+// file-scope device array, g_noalloc_scratch, of MUON_NOALLOC_SCRATCH_BYTES.
+// The CUDA runtime reserves it on every device where this library's kernels
+// are loaded, for the life of the process.  Host code must not pass the
+// array's name to a kernel (in host code it names a host-side stand-in); the
+// device address comes from cudaGetSymbolAddress, looked up once per device
+// with that device current, on the first call made on that device.  The host
+// side uses fixed-size static tables only.
 // ---------------------------------------------------------------------------
 namespace {
 
@@ -779,8 +771,9 @@ static __device__ __align__(256) unsigned char
 
 constexpr int kNoAllocMaxDevices = 64;
 constexpr int kNoAllocMaxItems = 8192;
-constexpr int kNoAllocMaxGramTiles = 4096;
-constexpr int kNoAllocMaxApplyTiles = 8192;
+constexpr int kNoAllocMaxSched = 65536;
+constexpr int kNoAllocMaxClusters = 1024;
+constexpr int kNoAllocMaxGroups = MUON_NOALLOC_MAX_MATS * kMaxNsSteps * 3;
 
 // Device address of g_noalloc_scratch per device (filled on first use).
 void* g_noalloc_dev_ptr[kNoAllocMaxDevices] = {};
@@ -791,28 +784,11 @@ std::mutex g_noalloc_mutex;
 Geom g_na_geom[MUON_NOALLOC_MAX_MATS];
 MatDev g_na_mats[MUON_NOALLOC_MAX_MATS];
 ProItem g_na_items[kNoAllocMaxItems];
-NsTile g_na_gram[kNoAllocMaxGramTiles];
-NsTile g_na_poly[kNoAllocMaxGramTiles];
-NsTile g_na_apply[kNoAllocMaxApplyTiles];
-
-NsTile g_na_tmp[kNoAllocMaxApplyTiles];
-
-// Tile order: longest K first, list order among equal K (the order the
-// plan's stable sort gives), without a heap buffer: one pass per distinct K
-// length, from the longest down.
-void sort_tiles_by_k(NsTile* v, int n) {
-  int out = 0;
-  int cur = 1 << 30;
-  while (out < n) {
-    int next = -1;
-    for (int i = 0; i < n; ++i)
-      if (v[i].kt < cur && v[i].kt > next) next = v[i].kt;
-    for (int i = 0; i < n; ++i)
-      if (v[i].kt == next) g_na_tmp[out++] = v[i];
-    cur = next;
-  }
-  std::memcpy(v, g_na_tmp, sizeof(NsTile) * n);
-}
+SchedMatrix g_na_smats[MUON_NOALLOC_MAX_MATS];
+SchedItem g_na_sched[kNoAllocMaxSched];
+SchedGroup g_na_groups[kNoAllocMaxGroups];
+int g_na_order[MUON_NOALLOC_MAX_MATS];
+double g_na_cltime[kNoAllocMaxClusters];
 
 }  // namespace
 
@@ -831,35 +807,16 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
 
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
 
-  // Geometry and lists into the fixed host tables.
+  // Geometry and work items into the fixed host tables.
   size_t off = 0;
-  int n_items = 0, n_gram = 0, n_apply = 0;
+  int n_items = 0;
   size_t pro_smem = 0;
   for (int i = 0; i < n_mats; ++i) {
-    const int rows = mats[i].rows, cols = mats[i].cols;
-    if (rows < 1 || cols < 1) return MUON_ERR_INVALID_ARG;
-    if (rows > (1 << 20) || cols > (1 << 20) ||
-        static_cast<long long>(rows) * cols > (1ll << 31) - 1)
-      return MUON_ERR_UNSUPPORTED;
     Geom& g = g_na_geom[i];
-    g.rows = rows;
-    g.cols = cols;
-    g.transposed = rows > cols;
-    g.m = std::min(rows, cols);
-    g.n = std::max(rows, cols);
-    g.ldx = static_cast<int>(align_up(g.n, 8));
-    g.lda = static_cast<int>(align_up(g.m, 8));
-    for (int b = 0; b < 2; ++b) {
-      g.x_off[b] = off;
-      off = align_up(off + static_cast<size_t>(g.m) * g.ldx * 2, 1024);
-    }
-    g.a_off = off;
-    off = align_up(off + static_cast<size_t>(g.m) * g.lda * 2, 1024);
-    g.b_off = off;
-    off = align_up(off + static_cast<size_t>(g.m) * g.lda * 2, 1024);
+    vs = layout_matrix(mats[i].rows, mats[i].cols, g, off);
+    if (vs != MUON_OK) return vs;
     vs = validate_matrix(mats[i], g);
     if (vs != MUON_OK) return vs;
-
     const int rt = pro_rows_per_item(g.rows, g.cols);
     g.part_first = n_items;
     for (int r0 = 0; r0 < g.rows; r0 += rt) {
@@ -869,41 +826,16 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
     g.part_count = n_items - g.part_first;
     if (g.transposed)
       pro_smem = std::max(pro_smem, static_cast<size_t>(rt) * (g.cols + 2) * 2);
-
-    const int gram_before = n_gram, apply_before = n_apply;
-    if (!append_pair_tiles(i, g, g_na_gram, g_na_poly, n_gram, kNoAllocMaxGramTiles,
-                           g_na_apply, n_apply, kNoAllocMaxApplyTiles))
-      return MUON_ERR_UNSUPPORTED;
-    g.n_sym_tiles = n_gram - gram_before;
-    g.n_apply_tiles = n_apply - apply_before;
+    fill_sched_matrix(g_na_smats[i], g);
   }
-  sort_tiles_by_k(g_na_gram, n_gram);
-  sort_tiles_by_k(g_na_poly, n_gram);
-  sort_tiles_by_k(g_na_apply, n_apply);
   const size_t part_off = off;
   off = align_up(off + static_cast<size_t>(n_items) * sizeof(float), 1024);
   const size_t scale_off = off;
   off = align_up(off + static_cast<size_t>(n_mats) * sizeof(float), 1024);
   const size_t counter_off = off;
-  const size_t counter_bytes =
-      static_cast<size_t>(n_mats) * (1 + 3 * std::max(ns_steps, 1)) * sizeof(int32_t);
+  const size_t counter_bytes = counter_bytes_for(n_mats, ns_steps);
   off = align_up(off + counter_bytes, 1024);
   const size_t ws_bytes = off;
-
-  // Layout of the device array: [error word][tables][workspace].
-  size_t t_off = 256;
-  const size_t mats_off = t_off;
-  t_off = align_up(t_off + sizeof(MatDev) * n_mats, 256);
-  const size_t items_off = t_off;
-  t_off = align_up(t_off + sizeof(ProItem) * n_items, 256);
-  const size_t gram_off = t_off;
-  t_off = align_up(t_off + sizeof(NsTile) * n_gram, 256);
-  const size_t poly_off = t_off;
-  t_off = align_up(t_off + sizeof(NsTile) * n_gram, 256);
-  const size_t apply_off = t_off;
-  t_off = align_up(t_off + sizeof(NsTile) * n_apply, 1024);
-  const size_t ws_off = t_off;
-  if (ws_off + ws_bytes > MUON_NOALLOC_SCRATCH_BYTES) return MUON_ERR_WORKSPACE;
 
   // Device address of the array on the current device (once per device).
   int dev = 0;
@@ -916,21 +848,33 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
       return MUON_ERR_CUDA;
     }
     const int clusters = query_max_clusters();
-    if (clusters <= 0) {
+    if (clusters <= 0 || clusters > kNoAllocMaxClusters) {
       cudaGetLastError();
       return MUON_ERR_CUDA;
     }
     g_noalloc_clusters[dev] = clusters;
     g_noalloc_dev_ptr[dev] = ptr;
   }
-  int num_sms = 148;
-  if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) !=
-      cudaSuccess)
-    return MUON_ERR_CUDA;
-  if (pro_smem > 48 * 1024 &&
-      cudaFuncSetAttribute(muon_prologue_kernel,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(pro_smem)) != cudaSuccess) {
+  const int clusters = g_noalloc_clusters[dev];
+  long long n_sched = 0;
+  if (ns_steps > 0) {
+    n_sched = build_schedule(g_na_smats, n_mats, ns_steps, clusters, g_na_sched,
+                             kNoAllocMaxSched, g_na_groups, g_na_order, g_na_cltime);
+    if (n_sched < 0) return MUON_ERR_UNSUPPORTED;
+  }
+
+  // Layout of the device array: [error word][tables][workspace].
+  size_t t_off = 256;
+  const size_t mats_off = t_off;
+  t_off = align_up(t_off + sizeof(MatDev) * n_mats, 256);
+  const size_t items_off = t_off;
+  t_off = align_up(t_off + sizeof(ProItem) * n_items, 256);
+  const size_t sched_off = t_off;
+  t_off = align_up(t_off + sizeof(SchedItem) * n_sched, 1024);
+  const size_t ws_off = t_off;
+  if (ws_off + ws_bytes > MUON_NOALLOC_SCRATCH_BYTES) return MUON_ERR_WORKSPACE;
+
+  if (!set_kernel_attributes(pro_smem)) {
     cudaGetLastError();
     return MUON_ERR_CUDA;
   }
@@ -943,29 +887,24 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // The array keeps the previous call's contents: the error word must start
-  // at zero; everything else is written before it is read.
+  // at zero (the counters are reset by the step itself); everything else is
+  // written before it is read.
   if (cudaMemsetAsync(base, 0, sizeof(int32_t), st) != cudaSuccess ||
       cudaMemcpyAsync(base + mats_off, g_na_mats, sizeof(MatDev) * n_mats,
                       cudaMemcpyHostToDevice, st) != cudaSuccess ||
       cudaMemcpyAsync(base + items_off, g_na_items, sizeof(ProItem) * n_items,
                       cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(base + gram_off, g_na_gram, sizeof(NsTile) * n_gram,
-                      cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(base + poly_off, g_na_poly, sizeof(NsTile) * n_gram,
-                      cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(base + apply_off, g_na_apply, sizeof(NsTile) * n_apply,
-                      cudaMemcpyHostToDevice, st) != cudaSuccess) {
+      (n_sched > 0 &&
+       cudaMemcpyAsync(base + sched_off, g_na_sched, sizeof(SchedItem) * n_sched,
+                       cudaMemcpyHostToDevice, st) != cudaSuccess)) {
     cudaGetLastError();
     return MUON_ERR_CUDA;
   }
 
   LaunchTables t{reinterpret_cast<const MatDev*>(base + mats_off),
                  reinterpret_cast<const ProItem*>(base + items_off), n_items,
-                 reinterpret_cast<const NsTile*>(base + gram_off), n_gram,
-                 reinterpret_cast<const NsTile*>(base + poly_off), n_gram,
-                 reinterpret_cast<const NsTile*>(base + apply_off), n_apply,
-                 reinterpret_cast<int32_t*>(base), num_sms, pro_smem,
-                 g_noalloc_clusters[dev]};
+                 reinterpret_cast<const SchedItem*>(base + sched_off), n_sched,
+                 reinterpret_cast<int32_t*>(base), pro_smem, clusters};
   StepScratch sc{reinterpret_cast<float*>(ws + part_off),
                  reinterpret_cast<float*>(ws + scale_off),
                  reinterpret_cast<int32_t*>(ws + counter_off), counter_bytes, n_mats};

@@ -57,6 +57,18 @@ struct NsTile {
   uint16_t kt;   // number of 64-wide K blocks
 };
 
+// One item of the persistent Newton-Schulz schedule: a pair tile of one
+// phase (gram, poly, apply) of one step of one matrix.
+struct SchedItem {
+  uint16_t mat;
+  uint16_t ti;    // pair-tile row (256 rows)
+  uint16_t tj;    // pair-tile column (256 columns)
+  uint16_t kt;    // number of 64-wide K blocks
+  uint8_t mode;   // kModeGram / kModePoly / kModeApply
+  uint8_t k;      // Newton-Schulz step
+  uint16_t pad;
+};
+
 struct HyperDev {
   float mu, lr, wd, eps_row, eps_frob;
   int32_t nesterov, eq_r;

@@ -1,0 +1,141 @@
+// Host-side schedule of the persistent Newton-Schulz kernel.
+//
+// The kernel runs a list of items (pair tiles of gram / poly / apply of every
+// step and matrix); cluster c executes list positions c, c + C, c + 2C, ...
+// in order and waits in-kernel until the phase an item reads is complete.
+// The order decides how often clusters stall, not correctness; every
+// dependency must precede its dependants (the kernel's deadlock-freedom
+// condition).  The order built here is phase-major: for each step the gram
+// tiles of all matrices, then the poly tiles, then the apply tiles, each
+// phase longest first (matrix order among equals).  A simulation of the
+// clusters under a simple cost model (tensor cycles per 64-deep K block plus
+// a fixed cost per item) gives its makespan; a greedy ready-first list
+// scheduler was tried under the same model and came out worse, because with
+// a fixed round-robin assignment an idle wait cannot be handed to another
+// cluster.  Uses only caller-provided arrays: no allocation.
+#pragma once
+
+#include <cstdint>
+
+#include "muon_types.cuh"
+
+namespace muonb200 {
+
+struct SchedMatrix {
+  int m, n;          // working shape
+  int t2;            // 256-row blocks of m
+  int tn;            // 256-column blocks of n
+};
+
+struct SchedGroup {
+  int mat, k, mode;
+  int size;          // tiles in this (matrix, step, phase)
+  int placed;
+  double done;       // simulated finish of the last placed tile
+  int dep;           // group whose completion this one reads, or -1
+};
+
+inline int sched_group_index(int mat, int k, int mode, int steps) {
+  return (mat * steps + k) * 3 + mode;
+}
+
+inline int sched_ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Item cost in tensor-core cycles of one CTA pair (256 x 256 x 64 per K
+// block) plus a fixed per-item cost; the last step's apply also moves W.
+inline double sched_cost(const SchedMatrix& mm, int mode, int k, int steps) {
+  const int kt = mode == kModeGram ? sched_ceil_div(mm.n, kTileK)
+                                   : sched_ceil_div(mm.m, kTileK);
+  double c = 512.0 * kt + 3000.0;
+  if (mode == kModeApply && k == steps - 1) c += 12000.0;
+  return c;
+}
+
+// Tile `idx` of a group: upper pair blocks for gram/poly, all blocks for apply.
+inline void sched_tile(const SchedMatrix& mm, int mode, int idx, int& ti, int& tj) {
+  if (mode == kModeApply) {
+    ti = idx / mm.tn;
+    tj = idx % mm.tn;
+    return;
+  }
+  int i = 0;
+  while (idx >= mm.t2 - i) {
+    idx -= mm.t2 - i;
+    ++i;
+  }
+  ti = i;
+  tj = i + idx;
+}
+
+// Returns the number of items written to `out` (capacity `cap`), or -1.
+// `groups` needs n_mats * steps * 3 entries, `order` (scratch) n_mats ints,
+// `cl_time` `clusters` doubles (the simulated finish time of each cluster).
+inline long long build_schedule(const SchedMatrix* mats, int n_mats, int steps,
+                                int clusters, SchedItem* out, long long cap,
+                                SchedGroup* groups, int* order, double* cl_time) {
+  long long total = 0;
+  for (int i = 0; i < n_mats; ++i)
+    for (int k = 0; k < steps; ++k)
+      for (int mode = 0; mode < 3; ++mode) {
+        SchedGroup& g = groups[sched_group_index(i, k, mode, steps)];
+        g.mat = i;
+        g.k = k;
+        g.mode = mode;
+        g.size = mode == kModeApply ? mats[i].t2 * mats[i].tn
+                                    : mats[i].t2 * (mats[i].t2 + 1) / 2;
+        g.placed = 0;
+        g.done = 0.0;
+        g.dep = mode == kModeGram ? (k == 0 ? -1 : sched_group_index(i, k - 1, kModeApply, steps))
+                                  : sched_group_index(i, k, mode - 1, steps);
+        total += g.size;
+      }
+  if (total > cap) return -1;
+  for (int c = 0; c < clusters; ++c) cl_time[c] = 0.0;
+
+  long long pos = 0;
+  for (int k = 0; k < steps; ++k)
+    for (int mode = 0; mode < 3; ++mode) {
+      // matrices of this phase, longest item first (insertion sort, stable)
+      for (int i = 0; i < n_mats; ++i) {
+        int j = i;
+        const double ci = sched_cost(mats[i], mode, k, steps);
+        while (j > 0 && sched_cost(mats[order[j - 1]], mode, k, steps) < ci) {
+          order[j] = order[j - 1];
+          --j;
+        }
+        order[j] = i;
+      }
+      // all tiles of one matrix consecutively, so that each matrix's phase
+      // completes as early as possible
+      for (int x = 0; x < n_mats; ++x) {
+        const int mi = order[x];
+        SchedGroup& g = groups[sched_group_index(mi, k, mode, steps)];
+        const SchedMatrix& mm = mats[mi];
+        const double dep_t = g.dep < 0 ? 0.0 : groups[g.dep].done;
+        const double cost = sched_cost(mm, mode, k, steps);
+        for (int t = 0; t < g.size; ++t) {
+          int ti = 0, tj = 0;
+          sched_tile(mm, mode, t, ti, tj);
+          SchedItem& it = out[pos];
+          it.mat = static_cast<uint16_t>(mi);
+          it.ti = static_cast<uint16_t>(ti);
+          it.tj = static_cast<uint16_t>(tj);
+          it.kt = static_cast<uint16_t>(mode == kModeGram ? sched_ceil_div(mm.n, kTileK)
+                                                           : sched_ceil_div(mm.m, kTileK));
+          it.mode = static_cast<uint8_t>(mode);
+          it.k = static_cast<uint8_t>(k);
+          it.pad = 0;
+          // simulation: in-order execution on cluster pos % clusters
+          const int c = static_cast<int>(pos % clusters);
+          const double start = cl_time[c] > dep_t ? cl_time[c] : dep_t;
+          cl_time[c] = start + cost;
+          g.placed += 1;
+          if (cl_time[c] > g.done) g.done = cl_time[c];
+          ++pos;
+        }
+      }
+    }
+  return pos;
+}
+
+}  // namespace muonb200

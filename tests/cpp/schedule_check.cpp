@@ -1,0 +1,42 @@
+// Host-side check of the Newton-Schulz list scheduler (schedule.h): reads
+// "n_mats steps clusters" then n_mats lines "rows cols" on stdin, builds the
+// schedule and prints one line per item "mat mode k ti tj kt", then
+// "makespan <simulated cycles>".
+#include <cstdio>
+#include <vector>
+
+#include "schedule.h"
+
+using namespace muonb200;
+
+int main() {
+  int n_mats = 0, steps = 0, clusters = 0;
+  if (std::scanf("%d %d %d", &n_mats, &steps, &clusters) != 3) return 2;
+  std::vector<SchedMatrix> mats(n_mats);
+  long long per_step = 0;
+  for (int i = 0; i < n_mats; ++i) {
+    int r = 0, c = 0;
+    if (std::scanf("%d %d", &r, &c) != 2) return 2;
+    SchedMatrix& s = mats[i];
+    s.m = r < c ? r : c;
+    s.n = r < c ? c : r;
+    s.t2 = (s.m + 255) / 256;
+    s.tn = (s.n + 255) / 256;
+    per_step += s.t2 * (s.t2 + 1) + s.t2 * s.tn;
+  }
+  std::vector<SchedItem> out(per_step * steps);
+  std::vector<SchedGroup> groups(static_cast<size_t>(n_mats) * steps * 3);
+  std::vector<int> order(n_mats);
+  std::vector<double> cl(clusters);
+  const long long n = build_schedule(mats.data(), n_mats, steps, clusters, out.data(),
+                                     static_cast<long long>(out.size()), groups.data(),
+                                     order.data(), cl.data());
+  if (n < 0) return 3;
+  for (long long i = 0; i < n; ++i)
+    std::printf("%d %d %d %d %d %d\n", out[i].mat, out[i].mode, out[i].k, out[i].ti,
+                out[i].tj, out[i].kt);
+  double mk = 0;
+  for (double t : cl) mk = t > mk ? t : mk;
+  std::printf("makespan %.0f\n", mk);
+  return 0;
+}
