@@ -10,7 +10,8 @@
 namespace muonb200 {
 
 constexpr int kEpiWarps = 8;                 // two per TMEM lane quadrant
-constexpr int kNsThreads = 64 + 32 * kEpiWarps;
+// producer warp, MMA warp, epilogue warps, completion-signal warp
+constexpr int kNsThreads = 96 + 32 * kEpiWarps;
 
 
 
@@ -37,5 +38,39 @@ __device__ __forceinline__ void load_row32_bf16(const __nv_bfloat16* src,
   }
 }
 
+// Row segment src[col0 .. col0 + 32) of a bf16 row as raw bf16 pairs (zeros
+// at and beyond `limit`); unpack_row32_bf16 widens it.
+__device__ __forceinline__ void load_row32_bf16_raw(const __nv_bfloat16* src,
+                                                    int col0, int limit,
+                                                    uint4 (&r)[4]) {
+  if (col0 + 32 <= limit) {
+    const uint4* p = reinterpret_cast<const uint4*>(src + col0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) r[q] = p[q];
+  } else {
+    const uint16_t* h = reinterpret_cast<const uint16_t*>(src);
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t lo = col0 + 2 * i < limit ? h[col0 + 2 * i] : 0u;
+      const uint32_t hi = col0 + 2 * i + 1 < limit ? h[col0 + 2 * i + 1] : 0u;
+      w[i] = lo | (hi << 16);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) r[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  }
+}
+
+__device__ __forceinline__ void unpack_row32_bf16(const uint4 (&r)[4], float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t w[4] = {r[q].x, r[q].y, r[q].z, r[q].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[8 * q + 2 * i] = __uint_as_float(w[i] << 16);
+      v[8 * q + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+}
 
 }  // namespace muonb200

@@ -75,7 +75,8 @@ struct MegaCfg {
   static constexpr int kTmemCols = 2 * kPairTile;
   static constexpr int kOutBlockElems = 32 * 32;
   static constexpr int kOutStageBytes = kEpiWarps * 2 * kOutBlockElems * 2;
-  static constexpr int kNumBars = 2 * kMegaStages + 7;
+  static constexpr int kEpiBars = 4;   // completion hand-off ring
+  static constexpr int kNumBars = 2 * kMegaStages + 5 + kEpiBars;
   static constexpr size_t kSmemBytes = 1024 +
       static_cast<size_t>(kMegaStages) * kStageBytes + kOutStageBytes +
       kNumBars * 8 + 16;
@@ -139,6 +140,107 @@ __device__ __forceinline__ const int32_t* dep_counter(const MegaParams& p,
   return done_counter(p, it.tl.mat, it.k, it.mode == kModePoly ? kModeGram : kModePoly);
 }
 
+// The fp32 weight update of the last step works on 32 x 32 blocks of the
+// working orientation (W itself, or W^T for transposed matrices), rows
+// row0 .. row0 + 32, columns col0 .. col0 + 32.  Full blocks of row-major W
+// with 16-byte rows are "coalesced": lane L holds rows row0 + 4 i + L / 8
+// (i = 0..7), columns col0 + 4 (L % 8) .. + 4, so each warp access covers
+// four whole 128-byte rows; O reaches that layout through the warp's shared
+// staging block.  Other blocks keep the accumulator's layout (lane = row).
+__device__ __forceinline__ bool w_block_coalesced(const MatDev* md, int row0, int col0) {
+  return !md->transposed && (md->n & 3) == 0 && col0 + 32 <= md->n &&
+         row0 + 32 <= md->m && (reinterpret_cast<uintptr_t>(md->w) & 15u) == 0 &&
+         (reinterpret_cast<uintptr_t>(md->out) & 15u) == 0;
+}
+
+// W of the block into wv (zeros outside the matrix).
+__device__ __forceinline__ void load_w_block(const MatDev* md, int row0, int col0,
+                                             int lane, float (&wv)[32]) {
+  const int m = md->m, n = md->n;
+  const float* __restrict__ w = md->w;
+  if (w_block_coalesced(md, row0, col0)) {
+    const float* base = w + static_cast<size_t>(row0 + (lane >> 3)) * n + col0 + 4 * (lane & 7);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 w4 = *reinterpret_cast<const float4*>(base + static_cast<size_t>(4 * i) * n);
+      wv[4 * i] = w4.x; wv[4 * i + 1] = w4.y; wv[4 * i + 2] = w4.z; wv[4 * i + 3] = w4.w;
+    }
+    return;
+  }
+  const int row = row0 + lane;
+  if (row >= m || col0 >= n) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) wv[e] = 0.f;
+    return;
+  }
+  if (!md->transposed) {
+    const float* w_row = w + static_cast<size_t>(row) * n + col0;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) wv[e] = col0 + e < n ? w_row[e] : 0.f;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      wv[e] = col0 + e < n ? w[static_cast<size_t>(col0 + e) * m + row] : 0.f;
+  }
+}
+
+// W <- W decay - step O on the block of load_w_block: wv holds its W, v the
+// accumulator row of this lane (O); O also goes to the optional update
+// output.  `stage` is the warp's 32 x 32 fp32 shared staging block.
+__device__ __forceinline__ void store_w_block(const MatDev* md, int row0, int col0,
+                                              int lane, float decay, float step,
+                                              const float (&wv)[32], const float (&v)[32],
+                                              float* stage) {
+  const int m = md->m, n = md->n;
+  float* __restrict__ w = md->w;
+  float* __restrict__ out = md->out;
+  if (w_block_coalesced(md, row0, col0)) {
+    // O row `lane` into the stage, 16-byte chunks XOR-swizzled by row so
+    // that both the row-wise writes and the transposed reads are free of
+    // bank conflicts.
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      *reinterpret_cast<float4*>(stage + lane * 32 + 4 * (q ^ (lane & 7))) =
+          make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    __syncwarp();
+    const int c = lane & 7;
+    const size_t g0 = static_cast<size_t>(row0 + (lane >> 3)) * n + col0 + 4 * c;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int rr = 4 * i + (lane >> 3);
+      const float4 o4 = *reinterpret_cast<const float4*>(stage + rr * 32 + 4 * (c ^ (rr & 7)));
+      const size_t g = g0 + static_cast<size_t>(4 * i) * n;
+      *reinterpret_cast<float4*>(w + g) =
+          make_float4(fmaf(wv[4 * i], decay, -step * o4.x),
+                      fmaf(wv[4 * i + 1], decay, -step * o4.y),
+                      fmaf(wv[4 * i + 2], decay, -step * o4.z),
+                      fmaf(wv[4 * i + 3], decay, -step * o4.w));
+      if (out) *reinterpret_cast<float4*>(out + g) = o4;
+    }
+    __syncwarp();
+    return;
+  }
+  const int row = row0 + lane;
+  if (row >= m || col0 >= n) return;
+  if (!md->transposed) {
+    const size_t g = static_cast<size_t>(row) * n + col0;
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      if (col0 + e < n) {
+        w[g + e] = fmaf(wv[e], decay, -step * v[e]);
+        if (out) out[g + e] = v[e];
+      }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      if (col0 + e < n) {
+        const size_t off = static_cast<size_t>(col0 + e) * m + row;
+        w[off] = fmaf(wv[e], decay, -step * v[e]);
+        if (out) out[off] = v[e];
+      }
+  }
+}
+
 __global__ void __launch_bounds__(kNsThreads, 1)
 ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
   using Cfg = MegaCfg;
@@ -149,9 +251,11 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
       reinterpret_cast<__nv_bfloat16*>(smem + kMegaStages * Cfg::kStageBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(
       smem + kMegaStages * Cfg::kStageBytes + Cfg::kOutStageBytes);
-  // bars: full[S], empty[S], tfull[2], tempty[2], drain, epi[2]
+  // bars: full[S], empty[S], tfull[2], tempty[2], drain, epi[kEpiBars]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // items whose completion the signal warp has published
+  volatile int* sig_count = reinterpret_cast<volatile int*>(tmem_slot + 2);
   constexpr int S = kMegaStages;
 
   const uint32_t smem0 = smem_addr(smem);
@@ -180,10 +284,11 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
       mbar_init(tempty_bar(a), 2 * kEpiWarps);
-      mbar_init(epi_bar(a), kEpiWarps);
     }
+    for (int a = 0; a < Cfg::kEpiBars; ++a) mbar_init(epi_bar(a), kEpiWarps);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
+    *sig_count = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -319,46 +424,75 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
       volatile int never = 0;
       mbar_wait_bounded(drain_bar, 0, &never, 10ull * 1000ull * 1000ull);
     }
-  } else {
+  } else if (warp < 2 + kEpiWarps) {
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;
     const int quad = warp & 3;
     const int half = ew >> 2;
     const int r_pair = static_cast<int>(rank) * 128 + quad * 32 + lane;
-    // This warp's 32 x 32 output block (row = lane) and its transpose.
+    // This warp's 32 x 32 bf16 staging block and its transpose (4 KB, also
+    // the fp32 staging block of the weight update).
     __nv_bfloat16* stg_d = out_stage + ew * 2 * Cfg::kOutBlockElems;
     __nv_bfloat16* stg_m = stg_d + Cfg::kOutBlockElems;
-    const uint32_t stg_d_addr = smem_addr(stg_d);
-    const uint32_t stg_m_addr = smem_addr(stg_m);
-    // Stages v (row `lane`) into the direct block and, if asked, the
-    // transposed block, then one lane issues the TMA stores.
-    auto put_block = [&](const CUtensorMap* tm, int row0_, int col0_, bool mirror,
-                         const float (&v)[32]) {
-      if (lane == 0) bulk_wait_group_read0();   // previous blocks read out
-      __syncwarp();
-      uint4* drow = reinterpret_cast<uint4*>(stg_d + lane * 32);
+    float* stage_f32 = reinterpret_cast<float*>(stg_d);
+    // Stores v (lane = row) as bf16 at rows row0_ .., columns col0_ .. of
+    // dst (leading dimension ld; rows below max_r, 8-column chunks starting
+    // below max_c, which ld covers) and, if `mirror`, its transpose at rows
+    // col0_ .., columns row0_ .. (square dst).  The block goes through shared
+    // memory so that every global store instruction writes eight whole
+    // 64-byte row segments; the 16-byte chunks of a staged row are
+    // XOR-swizzled by (row / 2) % 4, which keeps both the row writes and the
+    // segment reads free of bank conflicts.
+    auto put_block = [&](__nv_bfloat16* dst, int ld, int max_r, int max_c, int row0_,
+                         int col0_, bool mirror, const float (&v)[32]) {
+      uint4* srow = reinterpret_cast<uint4*>(stg_d) + lane * 4;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         __nv_bfloat162 h[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
           h[i] = __floats2bfloat162_rn(v[8 * q + 2 * i], v[8 * q + 2 * i + 1]);
-        drow[q] = *reinterpret_cast<uint4*>(h);
+        srow[q ^ ((lane >> 1) & 3)] = *reinterpret_cast<uint4*>(h);
       }
       if (mirror) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) stg_m[e * 32 + lane] = __float2bfloat16_rn(v[e]);
       }
-      fence_proxy_async_shared();
       __syncwarp();
-      if (lane == 0) {
-        tma_store_2d(tm, stg_d_addr, col0_, row0_);
-        if (mirror) tma_store_2d(tm, stg_m_addr, row0_, col0_);
-        bulk_commit_group();
+      const int c = lane & 3;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int rr = 8 * i + (lane >> 2);
+        const uint4 val = reinterpret_cast<const uint4*>(stg_d)[rr * 4 + (c ^ ((rr >> 1) & 3))];
+        const int gr = row0_ + rr, gc = col0_ + 8 * c;
+        if (gr < max_r && gc < max_c)
+          *reinterpret_cast<uint4*>(dst + static_cast<size_t>(gr) * ld + gc) = val;
       }
+      if (mirror) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int rr = 8 * i + (lane >> 2);
+          const uint4 val = reinterpret_cast<const uint4*>(stg_m)[rr * 4 + c];
+          const int gr = col0_ + rr, gc = row0_ + 8 * c;
+          if (gr < max_c && gc < max_r)
+            *reinterpret_cast<uint4*>(dst + static_cast<size_t>(gr) * ld + gc) = val;
+        }
+      }
+      __syncwarp();   // staging free for the next block
     };
     const uint32_t leader_tempty0 = mapa_shared(tempty_bar(0), 0);
-    const bool signaler = ew == 0 && lane == 0;
+    // Called after this warp's last accumulator read of an item: the leader
+    // may start the item after next in this accumulator while this one is
+    // still being stored.
+    auto release_acc = [&](int acc_) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(tempty_bar(acc_));
+        else mbar_arrive_cluster(leader_tempty0 + 8u * acc_);
+      }
+    };
+    constexpr int kLastCc = kPairTile / 32 - 2;   // cc of a warp's last block
     int lt = 0;
     for (int g = pair; g < total; g += npairs, ++lt) {
       const MegaItem item = mega_item(p, g);
@@ -366,6 +500,32 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
       const MatDev* md = p.mats + tl.mat;
       const int acc = lt & 1;
       const uint32_t aph = (lt >> 1) & 1;
+      const int row0 = tl.ti * kPairTile + static_cast<int>(rank) * 128 + quad * 32;
+      const int row = row0 + lane;
+      const int m = md->m;
+      const bool row_ok = row < m;
+      const bool first = item.k == 0;
+      const bool last = item.k == p.steps - 1;
+      const int colw = tl.tj * kPairTile + half * 32;   // this warp's first block
+      // Inputs that do not depend on the accumulator are requested before
+      // waiting for it: the last step's W blocks, the poly's rows of A.
+      float wa[32], wb[32];
+      uint4 ar0[4], ar1[4];
+      if (item.mode == kModeApply && last) {
+        load_w_block(md, row0, colw, lane, wa);
+        load_w_block(md, row0, colw + 64, lane, wb);
+      } else if (item.mode == kModePoly) {
+        // The generic reads of A need the gram stores of other CTAs.
+        if (lane == 0) {
+          int32_t target = 2 * md->n_sym_tiles;
+          if (!wait_count(done_counter(p, tl.mat, item.k, kModeGram), target,
+                          abort_flag, p.err))
+            fail(kErrTimeoutEpilogue);
+        }
+        __syncwarp();
+        if (row_ok)
+          load_row32_bf16_raw(md->a + static_cast<size_t>(row) * md->lda, colw, m, ar0);
+      }
       if (!mbar_wait_bounded(tfull_bar(acc), aph, abort_flag)) {
         fail(kErrTimeoutEpilogue);
         break;
@@ -373,153 +533,120 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * kPairTile);
-      const int row0 = tl.ti * kPairTile + static_cast<int>(rank) * 128 + quad * 32;
-      const int row = row0 + lane;
-      const int m = md->m;
-      const bool row_ok = row < m;
-      const bool first = item.k == 0;
-      const bool last = item.k == p.steps - 1;
       const float s = first ? p.mat_scale[tl.mat] : 1.f;
 
       if (item.mode == kModeGram || item.mode == kModePoly) {
         const bool diag_tile = tl.ti == tl.tj;
-        if (item.mode == kModePoly) {
-          // The generic reads of A below need the gram stores of other CTAs.
-          if (lane == 0) {
-            int32_t target = 2 * md->n_sym_tiles;
-            wait_count(done_counter(p, tl.mat, item.k, kModeGram), target,
-                       abort_flag, p.err);
-          }
-          __syncwarp();
-        }
-        const float pa = p.a[item.k], pb = p.b[item.k], pc = p.c[item.k];
-#pragma unroll 1
-        for (int cc = half; cc < kPairTile / 32; cc += 2) {
-          const int col0 = tl.tj * kPairTile + cc * 32;
-          float av[32];
-          if (item.mode == kModePoly && row_ok)
-            load_row32_bf16(md->a + static_cast<size_t>(row) * md->lda, col0, m, av);
+        const bool poly = item.mode == kModePoly;
+        // gram: s^2 X X^T;  poly: a I + b A + c A A (A A from the accumulator)
+        const float mul = poly ? p.c[item.k] : s * s;
+        const float pb = p.b[item.k];
+        const float pa = p.a[item.k];
+        // Block j (columns colw + 64 j) with A rows in `cur`; the next
+        // block's A rows are requested into `nxt` first.
+        auto block = [&](int j, const uint4 (&cur)[4], uint4 (&nxt)[4]) {
+          const int cc = half + 2 * j;
+          const int col0 = colw + 64 * j;
+          if (poly && j < 3 && row_ok)
+            load_row32_bf16_raw(md->a + static_cast<size_t>(row) * md->lda, col0 + 64, m, nxt);
           float v[32];
           tmem_load_32cols(tbase + cc * 32, v);
-          if (item.mode == kModeGram) {
-            const float s2 = s * s;
+          if (j == 3) release_acc(acc);
+          if (poly) {
+            float av[32];
+            unpack_row32_bf16(cur, av);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] *= s2;
-          } else if (row_ok) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = fmaf(pb, av[e], pc * v[e]);
+            for (int e = 0; e < 32; ++e) v[e] = row_ok ? fmaf(pb, av[e], mul * v[e]) : 0.f;
             if (diag_tile && (r_pair >> 5) == cc) {
               const int d = r_pair & 31;
 #pragma unroll
               for (int e = 0; e < 32; ++e)
                 if (e == d) v[e] += pa;
             }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] *= mul;
           }
-          put_block(item.mode == kModeGram ? &md->tm_as : &md->tm_bs, row0, col0,
-                    !diag_tile, v);
-        }
-      } else {
-        const int n = md->n;
-        const float decay = 1.f - p.lr * p.wd;
-        const float step = p.lr * md->update_scale;
-        const bool tr = md->transposed != 0;
+          put_block(poly ? md->b : md->a, md->lda, m, m, row0, col0, !diag_tile, v);
+        };
+        block(0, ar0, ar1);
+        block(1, ar1, ar0);
+        block(2, ar0, ar1);
+        block(3, ar1, ar0);
+      } else if (!last) {
 #pragma unroll 1
         for (int cc = half; cc < kPairTile / 32; cc += 2) {
           const int col0 = tl.tj * kPairTile + cc * 32;
-          const bool live = row_ok && col0 < n;
-          float wv[32];
-          float* w_row = nullptr;
-          const bool wvec = !tr && col0 + 32 <= n && (n & 3) == 0;
-          if (last && live) {
-            if (!tr) {
-              w_row = md->w + static_cast<size_t>(row) * n + col0;
-              if (wvec) {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                  const float4 w4 = reinterpret_cast<const float4*>(w_row)[q];
-                  wv[4 * q] = w4.x; wv[4 * q + 1] = w4.y;
-                  wv[4 * q + 2] = w4.z; wv[4 * q + 3] = w4.w;
-                }
-              } else {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) wv[e] = col0 + e < n ? w_row[e] : 0.f;
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                wv[e] = col0 + e < n
-                            ? md->w[static_cast<size_t>(col0 + e) * m + row] : 0.f;
-            }
-          }
           float v[32];
           tmem_load_32cols(tbase + cc * 32, v);
+          if (cc >= kLastCc) release_acc(acc);
           if (first) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] *= s;
           }
-          if (!last) {
-            // rows beyond m and columns beyond n are clipped by the TMA store
-            if (row0 < m && col0 < n)
-              put_block(&md->tm_xs[(item.k & 1) ^ 1], row0, col0, false, v);
-            continue;
-          }
-          if (!live) continue;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) wv[e] = fmaf(wv[e], decay, -step * v[e]);
-          if (!tr) {
-            float* o = md->out ? md->out + static_cast<size_t>(row) * n + col0 : nullptr;
-            if (wvec) {
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                reinterpret_cast<float4*>(w_row)[q] =
-                    make_float4(wv[4 * q], wv[4 * q + 1], wv[4 * q + 2], wv[4 * q + 3]);
-                if (o)
-                  reinterpret_cast<float4*>(o)[q] =
-                      make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (col0 + e < n) {
-                  w_row[e] = wv[e];
-                  if (o) o[e] = v[e];
-                }
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (col0 + e < n) {
-                const size_t off = static_cast<size_t>(col0 + e) * m + row;
-                md->w[off] = wv[e];
-                if (md->out) md->out[off] = v[e];
-              }
-          }
+          put_block(md->x[(item.k & 1) ^ 1], md->ldx, m, md->n, row0, col0, false, v);
         }
+      } else {
+        // W <- W (1 - lr wd) - lr scale O over this warp's four blocks; the
+        // next block's W is already in registers (loaded two blocks ahead,
+        // the first two before the accumulator was ready).
+        const float decay = 1.f - p.lr * p.wd;
+        const float step = p.lr * md->update_scale;
+        auto block = [&](int j, float (&wv)[32]) {
+          float v[32];
+          tmem_load_32cols(tbase + (half + 2 * j) * 32, v);
+          if (j == 3) release_acc(acc);
+          if (first) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] *= s;
+          }
+          store_w_block(md, row0, colw + 64 * j, lane, decay, step, wv, v, stage_f32);
+          if (j < 2) load_w_block(md, row0, colw + 64 * (j + 2), lane, wv);
+        };
+        block(0, wa);
+        block(1, wb);
+        block(2, wa);
+        block(3, wb);
       }
-      // Accumulator free: the leader may start the item after next.
-      tc_fence_before();
-      // This warp's stores of the item complete and visible (TMA readers
-      // too) before the item is counted.
-      if (lane == 0) bulk_wait_group0();
-      fence_proxy_async_global();
+      // Hand the item to the signal warp (the arrival releases this warp's
+      // stores to it).  Its barrier slot was last used four items ago; that
+      // item must have been published first, or the slot's phases would run
+      // ahead of the signal warp.
       __syncwarp();
+      bool ok = true;
       if (lane == 0) {
-        if (leader) mbar_arrive(tempty_bar(acc));
-        else mbar_arrive_cluster(leader_tempty0 + 8u * acc);
-        mbar_arrive(epi_bar(acc));
-      }
-      if (signaler) {
-        volatile int never = 0;
-        // all eight epilogue warps of this CTA have stored this item
-        if (mbar_wait_bounded(epi_bar(acc), aph, abort_flag)) {
-          __threadfence();
-          red_release_gpu_add(done_counter(p, tl.mat, item.k, item.mode), 1);
-        } else {
-          fail(kErrTimeoutEpilogue);
+        if (lt >= Cfg::kEpiBars) {
+          const uint64_t t0 = global_timer_ns();
+          while (*sig_count < lt - Cfg::kEpiBars + 1) {
+            if (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs) {
+              fail(kErrTimeoutEpilogue);
+              ok = false;
+              break;
+            }
+            __nanosleep(32);
+          }
         }
-        (void)never;
+        if (ok) mbar_arrive(epi_bar(lt % Cfg::kEpiBars));
       }
-      __syncwarp();
+      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+    }
+  } else {
+    // ------------------------------------------------------------ signal
+    // Publishes each item once all epilogue warps of this CTA have stored
+    // it: gpu-scope fence, then a release add on the item's phase counter.
+    if (lane == 0) {
+      int lt = 0;
+      for (int g = pair; g < total; g += npairs, ++lt) {
+        const MegaItem item = mega_item(p, g);
+        if (!mbar_wait_bounded(epi_bar(lt % Cfg::kEpiBars), (lt / Cfg::kEpiBars) & 1,
+                               abort_flag)) {
+          fail(kErrTimeoutEpilogue);
+          break;
+        }
+        __threadfence();
+        red_release_gpu_add(done_counter(p, item.tl.mat, item.k, item.mode), 1);
+        *sig_count = lt + 1;
+      }
     }
   }
 
