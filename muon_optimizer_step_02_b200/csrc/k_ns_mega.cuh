@@ -488,8 +488,8 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        if (leader) mbar_arrive(tempty_bar(acc_));
-        else mbar_arrive_cluster(leader_tempty0 + 8u * acc_);
+        if (leader) mbar_arrive_relaxed(tempty_bar(acc_));
+        else mbar_arrive_cluster_relaxed(leader_tempty0 + 8u * acc_);
       }
     };
     constexpr int kLastCc = kPairTile / 32 - 2;   // cc of a warp's last block
@@ -643,7 +643,8 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
           fail(kErrTimeoutEpilogue);
           break;
         }
-        __threadfence();
+        // release at gpu scope, cumulative over the stores the barrier
+        // made visible to this thread
         red_release_gpu_add(done_counter(p, item.tl.mat, item.k, item.mode), 1);
         *sig_count = lt + 1;
       }
