@@ -346,6 +346,9 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
         }
         const int arow = tl.ti * kPairTile + static_cast<int>(rank) * 128;
         const int bcol = tl.tj * kPairTile + static_cast<int>(rank) * 128;
+        // Diagonal tiles of X X^T and A A: this CTA's half of the B operand
+        // is the same 128 rows as its half of A, loaded once.
+        const bool same = item.mode != kModeApply && tl.ti == tl.tj;
         for (int kb = 0; kb < tl.kt; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
@@ -355,11 +358,12 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
             break;
           }
           if (p.fault == 1 && pair == 0 && it == 0 && leader) continue;  // test hook
-          if (leader) mbar_arrive_expect_tx(full_bar(s), Cfg::kTxBytes);
+          if (leader)
+            mbar_arrive_expect_tx(full_bar(s), same ? 2u * Cfg::kABytes : Cfg::kTxBytes);
           const uint32_t lfull = leader_full0 + 8u * s;
           tma_load_2d_pair(sA(s), tm_a, lfull, kb * kTileK, arow);
           if (item.mode != kModeApply) {
-            tma_load_2d_pair(sB(s), tm_b, lfull, kb * kTileK, bcol);
+            if (!same) tma_load_2d_pair(sB(s), tm_b, lfull, kb * kTileK, bcol);
           } else {
             tma_load_2d_pair(sB(s), tm_b, lfull, bcol, kb * kTileK);
             tma_load_2d_pair(sB(s) + 64 * kTileK * 2, tm_b, lfull, bcol + 64,
@@ -388,6 +392,7 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
       for (int g = pair; ok && g < total; g += npairs, ++lt) {
         const MegaItem item = mega_item(p, g);
         const bool bmn = item.mode == kModeApply;
+        const bool same = !bmn && item.tl.ti == item.tl.tj;   // B half = A half
         const uint32_t idesc = bmn ? idesc_mn : idesc_k;
         const int acc = lt & 1;
         const uint32_t aph = (lt >> 1) & 1;
@@ -412,7 +417,7 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
             const uint64_t adesc = smem_desc_sw128(sA(s) + kk * 32, 16, 1024);
             const uint64_t bdesc =
                 bmn ? smem_desc_sw128(sB(s) + kk * 2048, 64 * kTileK * 2, 1024)
-                    : smem_desc_sw128(sB(s) + kk * 32, 16, 1024);
+                    : smem_desc_sw128((same ? sA(s) : sB(s)) + kk * 32, 16, 1024);
             umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           umma_commit_pair_mc(empty_bar(s), 0x3);
