@@ -154,160 +154,171 @@ __device__ __forceinline__ void unpack_chunk(const ChunkRaw& c, float (&gv)[8],
 // (L2-resident), rebuilds U and writes the normalised row.  Keeping the row
 // out of registers keeps occupancy at three blocks (24 warps) per SM with
 // two chunks in flight per lane.
+//
+// Persistent: as many blocks as fit on the GPU at once, each taking the next
+// work item from `item_ctr` (items listed largest first) until none is left,
+// so that no partial last wave of blocks trails the pass.
 __global__ void __launch_bounds__(kProThreads, 3)
 muon_prologue_kernel(const MatDev* __restrict__ mats,
-                     const ProItem* __restrict__ items, HyperDev h,
+                     const ProItem* __restrict__ items, int n_items, HyperDev h,
                      float* __restrict__ partials, int32_t* __restrict__ tickets,
-                     float* __restrict__ mat_scale) {
+                     int32_t* __restrict__ item_ctr, float* __restrict__ mat_scale) {
   extern __shared__ __align__(16) unsigned char pro_smem[];
   __shared__ float warp_sums[kProThreads / 32];
   __shared__ int last_block;
+  __shared__ int cur_item;
 
-  const ProItem it = items[blockIdx.x];
-  const MatDev& md = mats[it.mat];
-  const int cols = md.cols;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool vec = (cols & 7) == 0;
-  const bool tr = md.transposed != 0;
-  const int sld = cols + 2;  // staging row stride (elements)
-  __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(pro_smem);
-  const int nch = (cols + 255) / 256;
-  const float mu = h.mu;
+  for (;;) {
+    __syncthreads();   // the previous item's staging and sums are consumed
+    if (threadIdx.x == 0) cur_item = atomicAdd(item_ctr, 1);
+    __syncthreads();
+    if (cur_item >= n_items) break;
+    const ProItem it = items[cur_item];
+    const MatDev& md = mats[it.mat];
+    const int cols = md.cols;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool vec = (cols & 7) == 0;
+    const bool tr = md.transposed != 0;
+    const int sld = cols + 2;  // staging row stride (elements)
+    __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(pro_smem);
+    const int nch = (cols + 255) / 256;
+    const float mu = h.mu;
 
-  float fro = 0.f;
-  for (int r = warp; r < it.nrows; r += kProThreads / 32) {
-    const int row = it.row0 + r;
-    const size_t base = static_cast<size_t>(row) * cols;
-    const uint16_t* __restrict__ g = md.g + base;
-    float* __restrict__ mo = md.mom + base;
-    __nv_bfloat16* xrow = tr ? nullptr : md.x[0] + static_cast<size_t>(row) * md.ldx;
-    __nv_bfloat16* srow = tr ? stage + r * sld : nullptr;
+    float fro = 0.f;
+    for (int r = warp; r < it.nrows; r += kProThreads / 32) {
+      const int row = it.row0 + r;
+      const size_t base = static_cast<size_t>(row) * cols;
+      const uint16_t* __restrict__ g = md.g + base;
+      float* __restrict__ mo = md.mom + base;
+      __nv_bfloat16* xrow = tr ? nullptr : md.x[0] + static_cast<size_t>(row) * md.ldx;
+      __nv_bfloat16* srow = tr ? stage + r * sld : nullptr;
 
-    // Pass 1: M' = mu M + G (stored), U = G + mu M', sum of U^2.
-    float ss = 0.f;
-    for (int c0 = 0; c0 < nch; c0 += kProBatch) {
-      if (vec) {
-        ChunkRaw raw[kProBatch];
-#pragma unroll
-        for (int b = 0; b < kProBatch; ++b) {
-          const int p0 = (c0 + b) * 256 + lane * 8;
-          if (c0 + b < nch && p0 < cols) load_chunk_vec(g, mo, p0, raw[b]);
-        }
-#pragma unroll
-        for (int b = 0; b < kProBatch; ++b) {
-          const int p0 = (c0 + b) * 256 + lane * 8;
-          if (c0 + b < nch && p0 < cols) {
+      // Pass 1: M' = mu M + G (stored), U = G + mu M', sum of U^2.
+      float ss = 0.f;
+      for (int c0 = 0; c0 < nch; c0 += kProBatch) {
+        if (vec) {
+          ChunkRaw raw[kProBatch];
+  #pragma unroll
+          for (int b = 0; b < kProBatch; ++b) {
+            const int p0 = (c0 + b) * 256 + lane * 8;
+            if (c0 + b < nch && p0 < cols) load_chunk_vec(g, mo, p0, raw[b]);
+          }
+  #pragma unroll
+          for (int b = 0; b < kProBatch; ++b) {
+            const int p0 = (c0 + b) * 256 + lane * 8;
+            if (c0 + b < nch && p0 < cols) {
+              float gv[8], mv[8];
+              unpack_chunk(raw[b], gv, mv);
+  #pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float mn = fmaf(mu, mv[e], gv[e]);
+                const float u = h.nesterov ? fmaf(mu, mn, gv[e]) : mn;
+                mv[e] = mn;
+                ss = fmaf(u, u, ss);
+              }
+              store_m(mo, true, c0 + b, lane, cols, mv);
+            }
+          }
+        } else {
+          for (int b = 0; b < kProBatch && c0 + b < nch; ++b) {
             float gv[8], mv[8];
-            unpack_chunk(raw[b], gv, mv);
-#pragma unroll
+            load_g_m(g, mo, false, c0 + b, lane, cols, gv, mv);
+  #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const float mn = fmaf(mu, mv[e], gv[e]);
               const float u = h.nesterov ? fmaf(mu, mn, gv[e]) : mn;
               mv[e] = mn;
               ss = fmaf(u, u, ss);
             }
-            store_m(mo, true, c0 + b, lane, cols, mv);
+            store_m(mo, false, c0 + b, lane, cols, mv);
           }
-        }
-      } else {
-        for (int b = 0; b < kProBatch && c0 + b < nch; ++b) {
-          float gv[8], mv[8];
-          load_g_m(g, mo, false, c0 + b, lane, cols, gv, mv);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float mn = fmaf(mu, mv[e], gv[e]);
-            const float u = h.nesterov ? fmaf(mu, mn, gv[e]) : mn;
-            mv[e] = mn;
-            ss = fmaf(u, u, ss);
-          }
-          store_m(mo, false, c0 + b, lane, cols, mv);
         }
       }
-    }
-    ss = warp_allreduce_sum(ss);
-    const float inv = h.eq_r ? 1.f / (sqrtf(ss) + h.eps_row) : 1.f;
-    fro += ss * inv * inv;
-    __syncwarp();  // this lane's M' stores precede its own re-reads below
+      ss = warp_allreduce_sum(ss);
+      const float inv = h.eq_r ? 1.f / (sqrtf(ss) + h.eps_row) : 1.f;
+      fro += ss * inv * inv;
+      __syncwarp();  // this lane's M' stores precede its own re-reads below
 
-    // Pass 2: U again from G and M', normalised, bf16.
-    for (int c0 = 0; c0 < nch; c0 += kProBatch) {
-      if (vec) {
-        ChunkRaw raw[kProBatch];
-#pragma unroll
-        for (int b = 0; b < kProBatch; ++b) {
-          const int p0 = (c0 + b) * 256 + lane * 8;
-          if (c0 + b < nch && p0 < cols) load_chunk_vec(g, mo, p0, raw[b]);
-        }
-#pragma unroll
-        for (int b = 0; b < kProBatch; ++b) {
-          const int p0 = (c0 + b) * 256 + lane * 8;
-          if (c0 + b < nch && p0 < cols) {
+      // Pass 2: U again from G and M', normalised, bf16.
+      for (int c0 = 0; c0 < nch; c0 += kProBatch) {
+        if (vec) {
+          ChunkRaw raw[kProBatch];
+  #pragma unroll
+          for (int b = 0; b < kProBatch; ++b) {
+            const int p0 = (c0 + b) * 256 + lane * 8;
+            if (c0 + b < nch && p0 < cols) load_chunk_vec(g, mo, p0, raw[b]);
+          }
+  #pragma unroll
+          for (int b = 0; b < kProBatch; ++b) {
+            const int p0 = (c0 + b) * 256 + lane * 8;
+            if (c0 + b < nch && p0 < cols) {
+              float gv[8], mv[8], x[8];
+              unpack_chunk(raw[b], gv, mv);
+  #pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float u = h.nesterov ? fmaf(mu, mv[e], gv[e]) : mv[e];
+                x[e] = u * inv;
+              }
+              emit_x(xrow, srow, tr, true, c0 + b, lane, cols, x);
+            }
+          }
+        } else {
+          for (int b = 0; b < kProBatch && c0 + b < nch; ++b) {
             float gv[8], mv[8], x[8];
-            unpack_chunk(raw[b], gv, mv);
-#pragma unroll
+            load_g_m(g, mo, false, c0 + b, lane, cols, gv, mv);
+  #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const float u = h.nesterov ? fmaf(mu, mv[e], gv[e]) : mv[e];
               x[e] = u * inv;
             }
-            emit_x(xrow, srow, tr, true, c0 + b, lane, cols, x);
+            emit_x(xrow, srow, tr, false, c0 + b, lane, cols, x);
           }
-        }
-      } else {
-        for (int b = 0; b < kProBatch && c0 + b < nch; ++b) {
-          float gv[8], mv[8], x[8];
-          load_g_m(g, mo, false, c0 + b, lane, cols, gv, mv);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float u = h.nesterov ? fmaf(mu, mv[e], gv[e]) : mv[e];
-            x[e] = u * inv;
-          }
-          emit_x(xrow, srow, tr, false, c0 + b, lane, cols, x);
         }
       }
     }
-  }
 
-  if (lane == 0) warp_sums[warp] = fro;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float s = 0.f;
-#pragma unroll
-    for (int w = 0; w < kProThreads / 32; ++w) s += warp_sums[w];
-    partials[blockIdx.x] = s;
-    // The last block of this matrix sums its partials in index order (the
-    // same order whichever block is last) into the Frobenius scale.
-    __threadfence();
-    const int ticket = atomicAdd(&tickets[it.mat], 1);
-    last_block = ticket == md.part_count - 1;
-  }
-  __syncthreads();
-  if (last_block && warp == 0) {
-    __threadfence();
-    float sum = 0.f;
-    if (lane == 0) {
-      const volatile float* pv = partials + md.part_first;
-      for (int i = 0; i < md.part_count; ++i) sum += pv[i];
-      mat_scale[it.mat] = 1.f / (sqrtf(sum) + h.eps_frob);
+    if (lane == 0) warp_sums[warp] = fro;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float s = 0.f;
+  #pragma unroll
+      for (int w = 0; w < kProThreads / 32; ++w) s += warp_sums[w];
+      partials[it.part] = s;
+      // The last block of this matrix sums its partials in index order (the
+      // same order whichever block is last) into the Frobenius scale.
+      __threadfence();
+      const int ticket = atomicAdd(&tickets[it.mat], 1);
+      last_block = ticket == md.part_count - 1;
     }
-  }
+    __syncthreads();
+    if (last_block && warp == 0) {
+      __threadfence();
+      float sum = 0.f;
+      if (lane == 0) {
+        const volatile float* pv = partials + md.part_first;
+        for (int i = 0; i < md.part_count; ++i) sum += pv[i];
+        mat_scale[it.mat] = 1.f / (sqrtf(sum) + h.eps_frob);
+      }
+    }
 
-  if (tr) {
-    // X[c][row0 + r] = stage[r][c]: 8 stored rows -> one 16-byte store.
-    const int ngrp = (it.nrows + 7) / 8;
-    __nv_bfloat16* xbase = md.x[0];
-    for (int idx = threadIdx.x; idx < cols * ngrp; idx += kProThreads) {
-      const int c = idx / ngrp;
-      const int grp = idx - c * ngrp;
-      const int r0 = grp * 8;
-      __nv_bfloat16* dst = xbase + static_cast<size_t>(c) * md.ldx + it.row0 + r0;
-      if (r0 + 8 <= it.nrows && ((it.row0 + r0) & 7) == 0) {
-        __align__(16) __nv_bfloat16 v[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) v[k] = stage[(r0 + k) * sld + c];
-        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(v);
-      } else {
-        for (int k = 0; k < 8 && r0 + k < it.nrows; ++k)
-          dst[k] = stage[(r0 + k) * sld + c];
+    if (tr) {
+      // X[c][row0 + r] = stage[r][c]: 8 stored rows -> one 16-byte store.
+      const int ngrp = (it.nrows + 7) / 8;
+      __nv_bfloat16* xbase = md.x[0];
+      for (int idx = threadIdx.x; idx < cols * ngrp; idx += kProThreads) {
+        const int c = idx / ngrp;
+        const int grp = idx - c * ngrp;
+        const int r0 = grp * 8;
+        __nv_bfloat16* dst = xbase + static_cast<size_t>(c) * md.ldx + it.row0 + r0;
+        if (r0 + 8 <= it.nrows && ((it.row0 + r0) & 7) == 0) {
+          __align__(16) __nv_bfloat16 v[8];
+  #pragma unroll
+          for (int k = 0; k < 8; ++k) v[k] = stage[(r0 + k) * sld + c];
+          *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(v);
+        } else {
+          for (int k = 0; k < 8 && r0 + k < it.nrows; ++k)
+            dst[k] = stage[(r0 + k) * sld + c];
+        }
       }
     }
   }

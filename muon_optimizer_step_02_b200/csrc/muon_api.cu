@@ -129,8 +129,33 @@ muon_status_t layout_matrix(int rows, int cols, Geom& g, size_t& off) {
 }
 
 size_t counter_bytes_for(int n_mats, int steps) {
-  // one prologue ticket per matrix + one count per (matrix, step, phase)
-  return static_cast<size_t>(n_mats) * (1 + 3 * std::max(steps, 1)) * sizeof(int32_t);
+  // the prologue's item counter, one prologue ticket per matrix, one count
+  // per (matrix, step, phase)
+  return (1 + static_cast<size_t>(n_mats) * (1 + 3 * std::max(steps, 1))) * sizeof(int32_t);
+}
+
+// Prologue work items, each with its partial-sum slot (the matrix's items
+// keep consecutive slots), listed largest first for the persistent prologue
+// (ties in slot order).  std::sort: no allocation.
+void order_prologue_items(ProItem* items, int n, const Geom* geom) {
+  std::sort(items, items + n, [geom](const ProItem& a, const ProItem& b) {
+    const long long wa = static_cast<long long>(a.nrows) * geom[a.mat].cols;
+    const long long wb = static_cast<long long>(b.nrows) * geom[b.mat].cols;
+    return wa != wb ? wa > wb : a.part < b.part;
+  });
+}
+
+// Blocks of the persistent prologue: all resident at once, at most one per item.
+int prologue_grid(int n_items, size_t pro_smem) {
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, muon_prologue_kernel, kProThreads,
+                                                    pro_smem) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return std::max(1, std::min(n_items, sms * std::max(per_sm, 1)));
 }
 
 struct TimingSlot {
@@ -158,6 +183,7 @@ struct muon_plan {
   size_t counter_off = 0;
   size_t counter_bytes = 0;
   size_t pro_smem = 0;
+  int pro_grid = 0;   // blocks of the persistent prologue
   int max_clusters = 0;
 
   // Newton-Schulz schedule for `sched_steps` steps (rebuilt when the step
@@ -238,6 +264,7 @@ struct LaunchTables {
   long long n_sched;
   int32_t* err;
   size_t pro_smem;
+  int pro_grid;       // blocks of the persistent prologue
   int clusters;       // clusters the schedule was built for (all resident)
 };
 
@@ -245,7 +272,7 @@ struct LaunchTables {
 struct StepScratch {
   float* partials;    // one per prologue item
   float* mat_scale;   // one per matrix
-  int32_t* counters;  // [tickets: n_mats][done: n_mats * K * 3], zeroed per step
+  int32_t* counters;  // [item counter][tickets: n_mats][done: n_mats * K * 3], zeroed per step
   size_t counter_bytes;
   int n_mats;
 };
@@ -381,12 +408,12 @@ void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
                   int fault, bool fresh, cudaStream_t st, Recorder* rec) {
   HyperDev hd{h.momentum, h.lr, h.weight_decay, h.eps_row, h.eps_frob,
               h.nesterov, h.eq_r};
-  int32_t* tickets = sc.counters;
-  int32_t* done = sc.counters + sc.n_mats;
+  int32_t* item_ctr = sc.counters;
+  int32_t* tickets = sc.counters + 1;
+  int32_t* done = sc.counters + 1 + sc.n_mats;
   cudaMemsetAsync(sc.counters, 0, sc.counter_bytes, st);
-  muon_prologue_kernel<<<static_cast<unsigned>(t.n_items), kProThreads,
-                         t.pro_smem, st>>>(t.mats, t.items, hd, sc.partials, tickets,
-                                           sc.mat_scale);
+  muon_prologue_kernel<<<static_cast<unsigned>(t.pro_grid), kProThreads, t.pro_smem, st>>>(
+      t.mats, t.items, t.n_items, hd, sc.partials, tickets, item_ctr, sc.mat_scale);
   if (rec) rec->after(MUON_KIND_PROLOGUE);
 
   if (ns_steps == 0) {
@@ -479,7 +506,8 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
     const int rt = pro_rows_per_item(g.rows, g.cols);
     g.part_first = static_cast<int>(plan->items.size());
     for (int r0 = 0; r0 < g.rows; r0 += rt)
-      plan->items.push_back(ProItem{i, r0, std::min(rt, g.rows - r0), 0});
+      plan->items.push_back(ProItem{i, r0, std::min(rt, g.rows - r0),
+                                    static_cast<int32_t>(plan->items.size())});
     g.part_count = static_cast<int>(plan->items.size()) - g.part_first;
     if (g.transposed)
       plan->pro_smem = std::max(plan->pro_smem,
@@ -488,6 +516,8 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
     per_step_items += 2 * g.n_sym_tiles + g.n_apply_tiles;
   }
   plan->sched_cap = per_step_items * std::max(max_ns_steps, 1);
+  order_prologue_items(plan->items.data(), static_cast<int>(plan->items.size()),
+                       plan->geom.data());
   if (plan->items.size() > 0x7FFFFFFF || plan->sched_cap > 0x7FFFFFFF) {
     delete plan;
     return MUON_ERR_UNSUPPORTED;
@@ -521,6 +551,8 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
   const size_t err_off = t_off;
   t_off += 256;
   if (plan->max_clusters <= 0 || !set_kernel_attributes(plan->pro_smem) ||
+      (plan->pro_grid = prologue_grid(static_cast<int>(plan->items.size()),
+                                      plan->pro_smem)) <= 0 ||
       cudaMalloc(&plan->d_block, t_off) != cudaSuccess) {
     cudaGetLastError();
     delete plan;
@@ -687,7 +719,7 @@ muon_status_t muon_step_batched(muon_plan_t* plan, const muon_matrix_t* mats,
   // ---- launches
   LaunchTables t{plan->d_mats, plan->d_items, static_cast<int>(plan->items.size()),
                  plan->d_sched, plan->sched_len, plan->d_err, plan->pro_smem,
-                 plan->max_clusters};
+                 plan->pro_grid, plan->max_clusters};
   StepScratch sc{reinterpret_cast<float*>(ws + plan->part_off),
                  reinterpret_cast<float*>(ws + plan->scale_off),
                  reinterpret_cast<int32_t*>(ws + plan->counter_off),
@@ -821,13 +853,15 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
     g.part_first = n_items;
     for (int r0 = 0; r0 < g.rows; r0 += rt) {
       if (n_items >= kNoAllocMaxItems) return MUON_ERR_UNSUPPORTED;
-      g_na_items[n_items++] = ProItem{i, r0, std::min(rt, g.rows - r0), 0};
+      g_na_items[n_items] = ProItem{i, r0, std::min(rt, g.rows - r0), n_items};
+      ++n_items;
     }
     g.part_count = n_items - g.part_first;
     if (g.transposed)
       pro_smem = std::max(pro_smem, static_cast<size_t>(rt) * (g.cols + 2) * 2);
     fill_sched_matrix(g_na_smats[i], g);
   }
+  order_prologue_items(g_na_items, n_items, g_na_geom);
   const size_t part_off = off;
   off = align_up(off + static_cast<size_t>(n_items) * sizeof(float), 1024);
   const size_t scale_off = off;
@@ -878,6 +912,8 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
     cudaGetLastError();
     return MUON_ERR_CUDA;
   }
+  const int pro_grid = prologue_grid(n_items, pro_smem);
+  if (pro_grid <= 0) return MUON_ERR_CUDA;
   char* base = static_cast<char*>(g_noalloc_dev_ptr[dev]);
   char* ws = base + ws_off;
   for (int i = 0; i < n_mats; ++i) {
@@ -904,7 +940,7 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
   LaunchTables t{reinterpret_cast<const MatDev*>(base + mats_off),
                  reinterpret_cast<const ProItem*>(base + items_off), n_items,
                  reinterpret_cast<const SchedItem*>(base + sched_off), n_sched,
-                 reinterpret_cast<int32_t*>(base), pro_smem, clusters};
+                 reinterpret_cast<int32_t*>(base), pro_smem, pro_grid, clusters};
   StepScratch sc{reinterpret_cast<float*>(ws + part_off),
                  reinterpret_cast<float*>(ws + scale_off),
                  reinterpret_cast<int32_t*>(ws + counter_off), counter_bytes, n_mats};

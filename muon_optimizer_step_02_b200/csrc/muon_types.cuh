@@ -46,7 +46,7 @@ struct ProItem {
   int32_t mat;
   int32_t row0;
   int32_t nrows;
-  int32_t pad;
+  int32_t part;          // slot of this item's Frobenius partial sum
 };
 
 // A tile of one tensor-core phase.
