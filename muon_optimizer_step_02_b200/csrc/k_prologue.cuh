@@ -148,23 +148,36 @@ __device__ __forceinline__ void unpack_chunk(const ChunkRaw& c, float (&gv)[8],
   mv[4] = c.m1.x; mv[5] = c.m1.y; mv[6] = c.m1.z; mv[7] = c.m1.w;
 }
 
-// One warp per stored row, two passes over the row with no register copy of
-// it: pass 1 streams G and M (kProBatch chunks of 8 elements per lane in
-// flight), writes M' and sums U^2; pass 2 re-reads G and the M' it just wrote
-// (L2-resident), rebuilds U and writes the normalised row.  Keeping the row
-// out of registers keeps occupancy at three blocks (24 warps) per SM with
-// two chunks in flight per lane.
+// Two variants, one launch each, over disjoint parts of the item list:
 //
-// Persistent: as many blocks as fit on the GPU at once, each taking the next
-// work item from `item_ctr` (items listed largest first) until none is left,
-// so that no partial last wave of blocks trails the pass.
-__global__ void __launch_bounds__(kProThreads, 3)
+// kOnePass (rows of up to kProOneWarps * 1024 elements, cols a multiple of 8;
+// every matrix of the 11L/16L/24L stacks): a row is spread over wpr warps of
+// 1024 elements each (four 8-element chunks per lane, all requested at once),
+// U stays in registers between the row-norm reduction and the write of X~,
+// and the row norm is summed across the row's warps in shared memory.  G and M
+// are read once: 12 bytes of HBM per element.
+//
+// two-pass (longer or unaligned rows): one warp per stored row and no
+// register copy of it.  Pass 1 streams G and M (kProBatch chunks of 8
+// elements per lane in flight), writes M' and sums U^2; pass 2 re-reads G and
+// the M' it just wrote (from L2 while the item is small enough), rebuilds U
+// and writes the normalised row.
+//
+// The variants are separate kernels because the one-pass register budget
+// (128 per thread at two blocks per SM) leaves no room for the other path's
+// live values, and the two-pass variant keeps three blocks per SM.  Both are persistent: as many blocks as fit on the GPU at
+// once, each taking the next work item from its own counter (items listed
+// largest first) until none is left, so that no partial last wave of blocks
+// trails the pass.
+template <bool kOnePass>
+__global__ void __launch_bounds__(kProThreads, kOnePass ? 2 : 3)
 muon_prologue_kernel(const MatDev* __restrict__ mats,
                      const ProItem* __restrict__ items, int n_items, HyperDev h,
                      float* __restrict__ partials, int32_t* __restrict__ tickets,
                      int32_t* __restrict__ item_ctr, float* __restrict__ mat_scale) {
   extern __shared__ __align__(16) unsigned char pro_smem[];
   __shared__ float warp_sums[kProThreads / 32];
+  __shared__ float row_sums[2][kProThreads / 32];
   __shared__ int last_block;
   __shared__ int cur_item;
 
@@ -185,93 +198,156 @@ muon_prologue_kernel(const MatDev* __restrict__ mats,
     const float mu = h.mu;
 
     float fro = 0.f;
-    for (int r = warp; r < it.nrows; r += kProThreads / 32) {
-      const int row = it.row0 + r;
-      const size_t base = static_cast<size_t>(row) * cols;
-      const uint16_t* __restrict__ g = md.g + base;
-      float* __restrict__ mo = md.mom + base;
-      __nv_bfloat16* xrow = tr ? nullptr : md.x[0] + static_cast<size_t>(row) * md.ldx;
-      __nv_bfloat16* srow = tr ? stage + r * sld : nullptr;
-
-      // Pass 1: M' = mu M + G (stored), U = G + mu M', sum of U^2.
-      float ss = 0.f;
-      for (int c0 = 0; c0 < nch; c0 += kProBatch) {
-        if (vec) {
-          ChunkRaw raw[kProBatch];
+    if constexpr (kOnePass) {
+      // warps per row: 1, 2, 4 or 8
+      const int wpr = cols <= 1024 ? 1 : cols <= 2048 ? 2 : cols <= 4096 ? 4 : 8;
+      const int rpp = (kProThreads / 32) / wpr;   // rows per pass of the block
+      const int rg = warp / wpr, wi = warp - rg * wpr;
+      for (int r0 = 0, pass = 0; r0 < it.nrows; r0 += rpp, ++pass) {
+        const int r = r0 + rg;
+        const bool act = r < it.nrows;
+        const int row = it.row0 + (act ? r : 0);
+        const size_t base = static_cast<size_t>(row) * cols;
+        const uint16_t* __restrict__ g = md.g + base;
+        float* __restrict__ mo = md.mom + base;
+        __nv_bfloat16* xrow = tr ? nullptr : md.x[0] + static_cast<size_t>(row) * md.ldx;
+        __nv_bfloat16* srow = tr ? stage + r * sld : nullptr;
+        ChunkRaw raw[4];
   #pragma unroll
-          for (int b = 0; b < kProBatch; ++b) {
-            const int p0 = (c0 + b) * 256 + lane * 8;
-            if (c0 + b < nch && p0 < cols) load_chunk_vec(g, mo, p0, raw[b]);
+        for (int j = 0; j < 4; ++j) {
+          const int p0 = (wi * 4 + j) * 256 + lane * 8;
+          if (act && p0 < cols) load_chunk_vec(g, mo, p0, raw[j]);
+        }
+        float u[4][8];
+        float ss = 0.f;
+  #pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int p0 = (wi * 4 + j) * 256 + lane * 8;
+          if (act && p0 < cols) {
+            float gv[8], mv[8];
+            unpack_chunk(raw[j], gv, mv);
+  #pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float mn = fmaf(mu, mv[e], gv[e]);
+              u[j][e] = h.nesterov ? fmaf(mu, mn, gv[e]) : mn;
+              mv[e] = mn;
+              ss = fmaf(u[j][e], u[j][e], ss);
+            }
+            store_m(mo, true, wi * 4 + j, lane, cols, mv);
           }
+        }
+        ss = warp_allreduce_sum(ss);
+        if (wpr > 1) {
+          // one barrier per pass; the two buffers alternate, so a buffer is
+          // rewritten only after every warp passed the next pass's barrier
+          if (lane == 0) row_sums[pass & 1][warp] = ss;
+          __syncthreads();
+          float t = 0.f;
+          for (int w = 0; w < wpr; ++w) t += row_sums[pass & 1][rg * wpr + w];
+          ss = t;
+        }
+        const float inv = h.eq_r ? 1.f / (sqrtf(ss) + h.eps_row) : 1.f;
+        if (act && wi == 0) fro += ss * inv * inv;
   #pragma unroll
-          for (int b = 0; b < kProBatch; ++b) {
-            const int p0 = (c0 + b) * 256 + lane * 8;
-            if (c0 + b < nch && p0 < cols) {
+        for (int j = 0; j < 4; ++j) {
+          const int p0 = (wi * 4 + j) * 256 + lane * 8;
+          if (act && p0 < cols) {
+            float x[8];
+  #pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = u[j][e] * inv;
+            emit_x(xrow, srow, tr, true, wi * 4 + j, lane, cols, x);
+          }
+        }
+      }
+    } else {
+      for (int r = warp; r < it.nrows; r += kProThreads / 32) {
+        const int row = it.row0 + r;
+        const size_t base = static_cast<size_t>(row) * cols;
+        const uint16_t* __restrict__ g = md.g + base;
+        float* __restrict__ mo = md.mom + base;
+        __nv_bfloat16* xrow = tr ? nullptr : md.x[0] + static_cast<size_t>(row) * md.ldx;
+        __nv_bfloat16* srow = tr ? stage + r * sld : nullptr;
+
+        // Pass 1: M' = mu M + G (stored), U = G + mu M', sum of U^2.
+        float ss = 0.f;
+        for (int c0 = 0; c0 < nch; c0 += kProBatch) {
+          if (vec) {
+            ChunkRaw raw[kProBatch];
+    #pragma unroll
+            for (int b = 0; b < kProBatch; ++b) {
+              const int p0 = (c0 + b) * 256 + lane * 8;
+              if (c0 + b < nch && p0 < cols) load_chunk_vec(g, mo, p0, raw[b]);
+            }
+    #pragma unroll
+            for (int b = 0; b < kProBatch; ++b) {
+              const int p0 = (c0 + b) * 256 + lane * 8;
+              if (c0 + b < nch && p0 < cols) {
+                float gv[8], mv[8];
+                unpack_chunk(raw[b], gv, mv);
+    #pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const float mn = fmaf(mu, mv[e], gv[e]);
+                  const float u = h.nesterov ? fmaf(mu, mn, gv[e]) : mn;
+                  mv[e] = mn;
+                  ss = fmaf(u, u, ss);
+                }
+                store_m(mo, true, c0 + b, lane, cols, mv);
+              }
+            }
+          } else {
+            for (int b = 0; b < kProBatch && c0 + b < nch; ++b) {
               float gv[8], mv[8];
-              unpack_chunk(raw[b], gv, mv);
-  #pragma unroll
+              load_g_m(g, mo, false, c0 + b, lane, cols, gv, mv);
+    #pragma unroll
               for (int e = 0; e < 8; ++e) {
                 const float mn = fmaf(mu, mv[e], gv[e]);
                 const float u = h.nesterov ? fmaf(mu, mn, gv[e]) : mn;
                 mv[e] = mn;
                 ss = fmaf(u, u, ss);
               }
-              store_m(mo, true, c0 + b, lane, cols, mv);
+              store_m(mo, false, c0 + b, lane, cols, mv);
             }
-          }
-        } else {
-          for (int b = 0; b < kProBatch && c0 + b < nch; ++b) {
-            float gv[8], mv[8];
-            load_g_m(g, mo, false, c0 + b, lane, cols, gv, mv);
-  #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float mn = fmaf(mu, mv[e], gv[e]);
-              const float u = h.nesterov ? fmaf(mu, mn, gv[e]) : mn;
-              mv[e] = mn;
-              ss = fmaf(u, u, ss);
-            }
-            store_m(mo, false, c0 + b, lane, cols, mv);
           }
         }
-      }
-      ss = warp_allreduce_sum(ss);
-      const float inv = h.eq_r ? 1.f / (sqrtf(ss) + h.eps_row) : 1.f;
-      fro += ss * inv * inv;
-      __syncwarp();  // this lane's M' stores precede its own re-reads below
+        ss = warp_allreduce_sum(ss);
+        const float inv = h.eq_r ? 1.f / (sqrtf(ss) + h.eps_row) : 1.f;
+        fro += ss * inv * inv;
+        __syncwarp();  // this lane's M' stores precede its own re-reads below
 
-      // Pass 2: U again from G and M', normalised, bf16.
-      for (int c0 = 0; c0 < nch; c0 += kProBatch) {
-        if (vec) {
-          ChunkRaw raw[kProBatch];
-  #pragma unroll
-          for (int b = 0; b < kProBatch; ++b) {
-            const int p0 = (c0 + b) * 256 + lane * 8;
-            if (c0 + b < nch && p0 < cols) load_chunk_vec(g, mo, p0, raw[b]);
-          }
-  #pragma unroll
-          for (int b = 0; b < kProBatch; ++b) {
-            const int p0 = (c0 + b) * 256 + lane * 8;
-            if (c0 + b < nch && p0 < cols) {
+        // Pass 2: U again from G and M', normalised, bf16.
+        for (int c0 = 0; c0 < nch; c0 += kProBatch) {
+          if (vec) {
+            ChunkRaw raw[kProBatch];
+    #pragma unroll
+            for (int b = 0; b < kProBatch; ++b) {
+              const int p0 = (c0 + b) * 256 + lane * 8;
+              if (c0 + b < nch && p0 < cols) load_chunk_vec(g, mo, p0, raw[b]);
+            }
+    #pragma unroll
+            for (int b = 0; b < kProBatch; ++b) {
+              const int p0 = (c0 + b) * 256 + lane * 8;
+              if (c0 + b < nch && p0 < cols) {
+                float gv[8], mv[8], x[8];
+                unpack_chunk(raw[b], gv, mv);
+    #pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const float u = h.nesterov ? fmaf(mu, mv[e], gv[e]) : mv[e];
+                  x[e] = u * inv;
+                }
+                emit_x(xrow, srow, tr, true, c0 + b, lane, cols, x);
+              }
+            }
+          } else {
+            for (int b = 0; b < kProBatch && c0 + b < nch; ++b) {
               float gv[8], mv[8], x[8];
-              unpack_chunk(raw[b], gv, mv);
-  #pragma unroll
+              load_g_m(g, mo, false, c0 + b, lane, cols, gv, mv);
+    #pragma unroll
               for (int e = 0; e < 8; ++e) {
                 const float u = h.nesterov ? fmaf(mu, mv[e], gv[e]) : mv[e];
                 x[e] = u * inv;
               }
-              emit_x(xrow, srow, tr, true, c0 + b, lane, cols, x);
+              emit_x(xrow, srow, tr, false, c0 + b, lane, cols, x);
             }
-          }
-        } else {
-          for (int b = 0; b < kProBatch && c0 + b < nch; ++b) {
-            float gv[8], mv[8], x[8];
-            load_g_m(g, mo, false, c0 + b, lane, cols, gv, mv);
-  #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float u = h.nesterov ? fmaf(mu, mv[e], gv[e]) : mv[e];
-              x[e] = u * inv;
-            }
-            emit_x(xrow, srow, tr, false, c0 + b, lane, cols, x);
           }
         }
       }

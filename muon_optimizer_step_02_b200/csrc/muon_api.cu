@@ -129,31 +129,40 @@ muon_status_t layout_matrix(int rows, int cols, Geom& g, size_t& off) {
 }
 
 size_t counter_bytes_for(int n_mats, int steps) {
-  // the prologue's item counter, one prologue ticket per matrix, one count
-  // per (matrix, step, phase)
-  return (1 + static_cast<size_t>(n_mats) * (1 + 3 * std::max(steps, 1))) * sizeof(int32_t);
+  // the two prologue item counters (one-pass, two-pass), one prologue ticket
+  // per matrix, one count per (matrix, step, phase)
+  return (2 + static_cast<size_t>(n_mats) * (1 + 3 * std::max(steps, 1))) * sizeof(int32_t);
 }
 
 // Prologue work items, each with its partial-sum slot (the matrix's items
-// keep consecutive slots), listed largest first for the persistent prologue
-// (ties in slot order).  std::sort: no allocation.
-void order_prologue_items(ProItem* items, int n, const Geom* geom) {
+// keep consecutive slots): the one-pass items first, then the two-pass ones,
+// each part listed largest first for its persistent kernel (ties in slot
+// order).  Returns the number of one-pass items.  std::sort: no allocation.
+int order_prologue_items(ProItem* items, int n, const Geom* geom) {
   std::sort(items, items + n, [geom](const ProItem& a, const ProItem& b) {
+    const bool oa = pro_one_pass(geom[a.mat].cols), ob = pro_one_pass(geom[b.mat].cols);
+    if (oa != ob) return oa;
     const long long wa = static_cast<long long>(a.nrows) * geom[a.mat].cols;
     const long long wb = static_cast<long long>(b.nrows) * geom[b.mat].cols;
     return wa != wb ? wa > wb : a.part < b.part;
   });
+  int n_one = 0;
+  while (n_one < n && pro_one_pass(geom[items[n_one].mat].cols)) ++n_one;
+  return n_one;
 }
 
-// Blocks of the persistent prologue: all resident at once, at most one per item.
+// Blocks of a persistent prologue kernel: all resident at once, at most one
+// per item (0 when there are no items).
+template <bool kOnePass>
 int prologue_grid(int n_items, size_t pro_smem) {
+  if (n_items <= 0) return 0;
   int dev = 0, sms = 0, per_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, muon_prologue_kernel, kProThreads,
-                                                    pro_smem) != cudaSuccess) {
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, muon_prologue_kernel<kOnePass>,
+                                                    kProThreads, pro_smem) != cudaSuccess) {
     cudaGetLastError();
-    return 0;
+    return -1;
   }
   return std::max(1, std::min(n_items, sms * std::max(per_sm, 1)));
 }
@@ -183,7 +192,8 @@ struct muon_plan {
   size_t counter_off = 0;
   size_t counter_bytes = 0;
   size_t pro_smem = 0;
-  int pro_grid = 0;   // blocks of the persistent prologue
+  int n_one = 0;       // one-pass prologue items (listed first)
+  int pro_grid[2] = {0, 0};   // blocks of the one-pass and two-pass prologues
   int max_clusters = 0;
 
   // Newton-Schulz schedule for `sched_steps` steps (rebuilt when the step
@@ -260,11 +270,12 @@ struct LaunchTables {
   const MatDev* mats;
   const ProItem* items;
   int n_items;
+  int n_one;          // one-pass prologue items (the first n_one of `items`)
   const SchedItem* sched;
   long long n_sched;
   int32_t* err;
   size_t pro_smem;
-  int pro_grid;       // blocks of the persistent prologue
+  int pro_grid[2];    // blocks of the one-pass and two-pass prologues
   int clusters;       // clusters the schedule was built for (all resident)
 };
 
@@ -272,7 +283,7 @@ struct LaunchTables {
 struct StepScratch {
   float* partials;    // one per prologue item
   float* mat_scale;   // one per matrix
-  int32_t* counters;  // [item counter][tickets: n_mats][done: n_mats * K * 3], zeroed per step
+  int32_t* counters;  // [item counters: 2][tickets: n_mats][done: n_mats * K * 3], zeroed per step
   size_t counter_bytes;
   int n_mats;
 };
@@ -355,9 +366,12 @@ bool set_kernel_attributes(size_t pro_smem) {
                            static_cast<int>(kMegaSmemBytes)) != cudaSuccess)
     return false;
   if (pro_smem > 48 * 1024 &&
-      cudaFuncSetAttribute(muon_prologue_kernel,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(pro_smem)) != cudaSuccess)
+      (cudaFuncSetAttribute(muon_prologue_kernel<true>,
+                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            static_cast<int>(pro_smem)) != cudaSuccess ||
+       cudaFuncSetAttribute(muon_prologue_kernel<false>,
+                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            static_cast<int>(pro_smem)) != cudaSuccess))
     return false;
   return true;
 }
@@ -409,11 +423,18 @@ void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
   HyperDev hd{h.momentum, h.lr, h.weight_decay, h.eps_row, h.eps_frob,
               h.nesterov, h.eq_r};
   int32_t* item_ctr = sc.counters;
-  int32_t* tickets = sc.counters + 1;
-  int32_t* done = sc.counters + 1 + sc.n_mats;
+  int32_t* tickets = sc.counters + 2;
+  int32_t* done = sc.counters + 2 + sc.n_mats;
   cudaMemsetAsync(sc.counters, 0, sc.counter_bytes, st);
-  muon_prologue_kernel<<<static_cast<unsigned>(t.pro_grid), kProThreads, t.pro_smem, st>>>(
-      t.mats, t.items, t.n_items, hd, sc.partials, tickets, item_ctr, sc.mat_scale);
+  if (t.n_one > 0)
+    muon_prologue_kernel<true><<<static_cast<unsigned>(t.pro_grid[0]), kProThreads,
+                                 t.pro_smem, st>>>(
+        t.mats, t.items, t.n_one, hd, sc.partials, tickets, item_ctr, sc.mat_scale);
+  if (t.n_items > t.n_one)
+    muon_prologue_kernel<false><<<static_cast<unsigned>(t.pro_grid[1]), kProThreads,
+                                  t.pro_smem, st>>>(
+        t.mats, t.items + t.n_one, t.n_items - t.n_one, hd, sc.partials, tickets,
+        item_ctr + 1, sc.mat_scale);
   if (rec) rec->after(MUON_KIND_PROLOGUE);
 
   if (ns_steps == 0) {
@@ -516,8 +537,9 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
     per_step_items += 2 * g.n_sym_tiles + g.n_apply_tiles;
   }
   plan->sched_cap = per_step_items * std::max(max_ns_steps, 1);
-  order_prologue_items(plan->items.data(), static_cast<int>(plan->items.size()),
-                       plan->geom.data());
+  plan->n_one = order_prologue_items(plan->items.data(),
+                                     static_cast<int>(plan->items.size()),
+                                     plan->geom.data());
   if (plan->items.size() > 0x7FFFFFFF || plan->sched_cap > 0x7FFFFFFF) {
     delete plan;
     return MUON_ERR_UNSUPPORTED;
@@ -550,9 +572,10 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
   t_off = align_up(t_off + sizeof(SchedItem) * plan->sched_cap, 256);
   const size_t err_off = t_off;
   t_off += 256;
+  const int n_two = static_cast<int>(plan->items.size()) - plan->n_one;
   if (plan->max_clusters <= 0 || !set_kernel_attributes(plan->pro_smem) ||
-      (plan->pro_grid = prologue_grid(static_cast<int>(plan->items.size()),
-                                      plan->pro_smem)) <= 0 ||
+      (plan->pro_grid[0] = prologue_grid<true>(plan->n_one, plan->pro_smem)) < 0 ||
+      (plan->pro_grid[1] = prologue_grid<false>(n_two, plan->pro_smem)) < 0 ||
       cudaMalloc(&plan->d_block, t_off) != cudaSuccess) {
     cudaGetLastError();
     delete plan;
@@ -718,8 +741,8 @@ muon_status_t muon_step_batched(muon_plan_t* plan, const muon_matrix_t* mats,
 
   // ---- launches
   LaunchTables t{plan->d_mats, plan->d_items, static_cast<int>(plan->items.size()),
-                 plan->d_sched, plan->sched_len, plan->d_err, plan->pro_smem,
-                 plan->pro_grid, plan->max_clusters};
+                 plan->n_one, plan->d_sched, plan->sched_len, plan->d_err, plan->pro_smem,
+                 {plan->pro_grid[0], plan->pro_grid[1]}, plan->max_clusters};
   StepScratch sc{reinterpret_cast<float*>(ws + plan->part_off),
                  reinterpret_cast<float*>(ws + plan->scale_off),
                  reinterpret_cast<int32_t*>(ws + plan->counter_off),
@@ -861,7 +884,7 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
       pro_smem = std::max(pro_smem, static_cast<size_t>(rt) * (g.cols + 2) * 2);
     fill_sched_matrix(g_na_smats[i], g);
   }
-  order_prologue_items(g_na_items, n_items, g_na_geom);
+  const int n_one = order_prologue_items(g_na_items, n_items, g_na_geom);
   const size_t part_off = off;
   off = align_up(off + static_cast<size_t>(n_items) * sizeof(float), 1024);
   const size_t scale_off = off;
@@ -912,8 +935,9 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
     cudaGetLastError();
     return MUON_ERR_CUDA;
   }
-  const int pro_grid = prologue_grid(n_items, pro_smem);
-  if (pro_grid <= 0) return MUON_ERR_CUDA;
+  const int pro_grid_one = prologue_grid<true>(n_one, pro_smem);
+  const int pro_grid_two = prologue_grid<false>(n_items - n_one, pro_smem);
+  if (pro_grid_one < 0 || pro_grid_two < 0) return MUON_ERR_CUDA;
   char* base = static_cast<char*>(g_noalloc_dev_ptr[dev]);
   char* ws = base + ws_off;
   for (int i = 0; i < n_mats; ++i) {
@@ -938,9 +962,10 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
   }
 
   LaunchTables t{reinterpret_cast<const MatDev*>(base + mats_off),
-                 reinterpret_cast<const ProItem*>(base + items_off), n_items,
+                 reinterpret_cast<const ProItem*>(base + items_off), n_items, n_one,
                  reinterpret_cast<const SchedItem*>(base + sched_off), n_sched,
-                 reinterpret_cast<int32_t*>(base), pro_smem, pro_grid, clusters};
+                 reinterpret_cast<int32_t*>(base), pro_smem, {pro_grid_one, pro_grid_two},
+                 clusters};
   StepScratch sc{reinterpret_cast<float*>(ws + part_off),
                  reinterpret_cast<float*>(ws + scale_off),
                  reinterpret_cast<int32_t*>(ws + counter_off), counter_bytes, n_mats};

@@ -13,6 +13,13 @@ constexpr int kPairTile = 256;    // CTA-pair tile: 256 rows (128 per CTA) x 256
 constexpr int kProRows = 32;      // rows per prologue work item
 constexpr int kProThreads = 256;  // 8 warps
 constexpr int kProBatch = 2;      // row chunks (of 256 elements) in flight per warp
+constexpr int kProOneWarps = 8;   // one-pass rows: up to 8 warps x 1024 elements
+
+// Stored rows that the one-pass prologue takes: a multiple of 8 elements (one
+// 16-byte load of G per chunk) and at most kProOneWarps * 1024 elements.
+__host__ __device__ constexpr bool pro_one_pass(int cols) {
+  return (cols & 7) == 0 && cols <= kProOneWarps * 1024;
+}
 
 // Per-matrix record.  Tensor maps first (64-byte aligned), pointers after.
 struct alignas(64) MatDev {

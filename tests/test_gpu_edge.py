@@ -36,6 +36,30 @@ def test_ragged_batch_in_one_plan():
         check_step(g, step, list(range(w.n_mats)))
 
 
+# Row lengths that select each prologue variant: one-pass rows spread over 1,
+# 2, 4 and 8 warps (cols a multiple of 8, at most 8192), rows too long for it
+# (8200, 8-aligned) and unaligned long rows (8201); the transposed write-out
+# with a row over two warps.
+PROLOGUE_ROWS = [(24, 1000), (40, 3000), (24, 6000), (16, 8192), (9, 8200),
+                 (12, 8201), (1100, 1040)]
+
+
+@pytest.mark.parametrize("shape", PROLOGUE_ROWS, ids=lambda s: f"{s[0]}x{s[1]}")
+def test_prologue_row_lengths(shape):
+    w = wl.custom([shape], H, Q5, grad_std=1.0, wid=110)
+    g = GpuMuon(w)
+    for step in range(2):
+        check_step(g, step, [0])
+
+
+def test_prologue_variants_in_one_plan():
+    """One-pass and two-pass prologue items in the same step."""
+    w = wl.custom(PROLOGUE_ROWS, H, Q5, grad_std=1.0, wid=111)
+    g = GpuMuon(w)
+    for step in range(2):
+        check_step(g, step, list(range(w.n_mats)))
+
+
 @pytest.mark.parametrize("k", [1, 2, 4, 5])
 def test_step_counts(k):
     w = wl.custom([(256, 512), (512, 256), (200, 136)], H, Q5[:k], wid=102)
