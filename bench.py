@@ -197,7 +197,7 @@ class Workload:
             self._ema()
 
     def launches_per_step(self) -> int:
-        n = self.B.step_launches(len(self.w.coeffs))
+        n = self.plan.step_launches(len(self.w.coeffs))
         if self.w.ema_decay is not None:
             n += self.B.ema_launches(len(self.E))
         return n

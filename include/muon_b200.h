@@ -163,8 +163,13 @@ muon_status_t muon_plan_set_timing(muon_plan_t *plan, int32_t enable);
 muon_status_t muon_plan_timing_read(muon_plan_t *plan, int32_t *launches,
                                     double *ms, int32_t n_kinds);
 
-/* Kernel launches of one call with ns_steps steps (for launch accounting). */
+/* Kernel launches of one call with ns_steps steps (for launch accounting):
+ * muon_step_launches counts a plan whose rows all take the same prologue
+ * kernel (one-pass: row length a multiple of 8 and at most 8192; two-pass
+ * otherwise); muon_plan_step_launches counts the given plan exactly (0 for
+ * a null plan or negative ns_steps). */
 int32_t muon_step_launches(int32_t ns_steps);
+int32_t muon_plan_step_launches(const muon_plan_t *plan, int32_t ns_steps);
 int32_t ema_update_launches(int32_t n_tensors);
 
 /* Test hook: fault 1 makes the tensor-core kernel's load warp skip one

@@ -86,6 +86,8 @@ def lib():
     L.muon_plan_timing_read.restype = c_int32
     L.muon_step_launches.argtypes = [c_int32]
     L.muon_step_launches.restype = c_int32
+    L.muon_plan_step_launches.argtypes = [c_void_p, c_int32]
+    L.muon_plan_step_launches.restype = c_int32
     L.ema_update_launches.argtypes = [c_int32]
     L.ema_update_launches.restype = c_int32
     L.muon_plan_set_fault.argtypes = [c_void_p, c_int32]
@@ -216,6 +218,9 @@ class MuonPlan:
 
     def last_error(self, stream=None) -> int:
         return int(lib().muon_get_last_error(self._h, _stream_handle(stream)))
+
+    def step_launches(self, ns_steps: int) -> int:
+        return int(lib().muon_plan_step_launches(self._h, int(ns_steps)))
 
     def set_timing(self, enable: bool):
         _check(lib().muon_plan_set_timing(self._h, int(enable)),

@@ -5,9 +5,9 @@
 // working orientation (transposed through shared memory when rows > cols);
 // the Frobenius partial sum of X~ over the work item goes to `partials`.
 //
-// The Frobenius scale s = 1 / (||X~||_F + eps_frob) of each matrix is also
-// finished here: every block writes its partial sum, and the last block of a
-// matrix (ticket counter) adds the matrix's partials in index order.
+// Every work item writes its Frobenius partial sum to its own slot; the
+// scale s = 1 / (||X~||_F + eps_frob) of each matrix is summed from them by
+// muon_frob_scale_kernel (one warp per matrix, a fixed order).
 //
 // Sources: PR #1893 "Record: L_ParallelResiduals_UNetSkips_DepthRecur_Muon_
 // 1.0901", table "Architecture and training stack", row "Optimizer" (Muon,
@@ -173,20 +173,19 @@ template <bool kOnePass>
 __global__ void __launch_bounds__(kProThreads, kOnePass ? 2 : 3)
 muon_prologue_kernel(const MatDev* __restrict__ mats,
                      const ProItem* __restrict__ items, int n_items, HyperDev h,
-                     float* __restrict__ partials, int32_t* __restrict__ tickets,
-                     int32_t* __restrict__ item_ctr, float* __restrict__ mat_scale) {
+                     float* __restrict__ partials, int32_t* __restrict__ item_ctr) {
   extern __shared__ __align__(16) unsigned char pro_smem[];
   __shared__ float warp_sums[kProThreads / 32];
   __shared__ float row_sums[2][kProThreads / 32];
-  __shared__ int last_block;
   __shared__ int cur_item;
 
   for (;;) {
     __syncthreads();   // the previous item's staging and sums are consumed
     if (threadIdx.x == 0) cur_item = atomicAdd(item_ctr, 1);
     __syncthreads();
-    if (cur_item >= n_items) break;
-    const ProItem it = items[cur_item];
+    const int idx = cur_item;
+    if (idx >= n_items) break;
+    const ProItem it = items[idx];
     const MatDev& md = mats[it.mat];
     const int cols = md.cols;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -200,7 +199,7 @@ muon_prologue_kernel(const MatDev* __restrict__ mats,
     float fro = 0.f;
     if constexpr (kOnePass) {
       // warps per row: 1, 2, 4 or 8
-      const int wpr = cols <= 1024 ? 1 : cols <= 2048 ? 2 : cols <= 4096 ? 4 : 8;
+      const int wpr = pro_warps_per_row(cols);
       const int rpp = (kProThreads / 32) / wpr;   // rows per pass of the block
       const int rg = warp / wpr, wi = warp - rg * wpr;
       for (int r0 = 0, pass = 0; r0 < it.nrows; r0 += rpp, ++pass) {
@@ -359,22 +358,7 @@ muon_prologue_kernel(const MatDev* __restrict__ mats,
       float s = 0.f;
   #pragma unroll
       for (int w = 0; w < kProThreads / 32; ++w) s += warp_sums[w];
-      partials[it.part] = s;
-      // The last block of this matrix sums its partials in index order (the
-      // same order whichever block is last) into the Frobenius scale.
-      __threadfence();
-      const int ticket = atomicAdd(&tickets[it.mat], 1);
-      last_block = ticket == md.part_count - 1;
-    }
-    __syncthreads();
-    if (last_block && warp == 0) {
-      __threadfence();
-      float sum = 0.f;
-      if (lane == 0) {
-        const volatile float* pv = partials + md.part_first;
-        for (int i = 0; i < md.part_count; ++i) sum += pv[i];
-        mat_scale[it.mat] = 1.f / (sqrtf(sum) + h.eps_frob);
-      }
+      partials[it.part] = s;   // summed per matrix by muon_frob_scale_kernel
     }
 
     if (tr) {
@@ -398,6 +382,23 @@ muon_prologue_kernel(const MatDev* __restrict__ mats,
       }
     }
   }
+}
+
+// The Frobenius scale s = 1 / (||X~||_F + eps_frob) of every matrix from its
+// prologue partials: one warp per matrix, lane l adds slots l, l + 32, ...
+// and the warp's butterfly adds the lanes, the same order on every run.
+__global__ void __launch_bounds__(256)
+muon_frob_scale_kernel(const MatDev* __restrict__ mats, int n_mats,
+                       const float* __restrict__ partials, float eps_frob,
+                       float* __restrict__ mat_scale) {
+  const int mat = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (mat >= n_mats) return;
+  const MatDev& md = mats[mat];
+  float s = 0.f;
+  for (int i = lane; i < md.part_count; i += 32) s += partials[md.part_first + i];
+  s = warp_allreduce_sum(s);
+  if (lane == 0) mat_scale[mat] = 1.f / (sqrtf(s) + eps_frob);
 }
 
 // ns_steps == 0: O = s X~ straight from the prologue's output, then the

@@ -21,6 +21,7 @@
 
 #include "muon_b200.h"
 
+
 #include "k_ema.cuh"
 #include "k_ns_mega.cuh"
 #include "k_prologue.cuh"
@@ -91,12 +92,23 @@ struct Geom {
   int n_sym_tiles, n_apply_tiles;  // pair tiles per phase
 };
 
+// Stored rows per prologue work item.  A transposed item is staged in shared
+// memory whole: up to kProSmemCap in the two-pass kernel (three blocks per
+// SM), up to kProTransBufCap in the one-pass kernel (two blocks per SM).
 int pro_rows_per_item(int rows, int cols) {
   if (rows <= cols) return kProRows;
-  size_t per_row = static_cast<size_t>(cols + 2) * 2;
-  int rt = static_cast<int>(std::min<size_t>(kProRows, kProSmemCap / per_row));
+  const size_t cap = pro_one_pass(cols) ? kProTransBufCap : kProSmemCap;
+  const size_t per_row = static_cast<size_t>(cols + 2) * 2;
+  int rt = static_cast<int>(std::min<size_t>(kProRows, cap / per_row));
   if (rt >= 8) rt &= ~7;
   return std::max(rt, 1);
+}
+
+// Shared memory of one transposed staging buffer of the matrix (0 when the
+// matrix is not transposed).
+size_t pro_trans_bytes(int rows, int cols) {
+  if (rows <= cols) return 0;
+  return static_cast<size_t>(pro_rows_per_item(rows, cols)) * (cols + 2) * 2;
 }
 
 // Shape checks, geometry, and the workspace offsets of X ping/pong, A, B'.
@@ -129,9 +141,9 @@ muon_status_t layout_matrix(int rows, int cols, Geom& g, size_t& off) {
 }
 
 size_t counter_bytes_for(int n_mats, int steps) {
-  // the two prologue item counters (one-pass, two-pass), one prologue ticket
-  // per matrix, one count per (matrix, step, phase)
-  return (2 + static_cast<size_t>(n_mats) * (1 + 3 * std::max(steps, 1))) * sizeof(int32_t);
+  // the two prologue item counters (one-pass, two-pass), one count per
+  // (matrix, step, phase)
+  return (2 + static_cast<size_t>(n_mats) * 3 * std::max(steps, 1)) * sizeof(int32_t);
 }
 
 // Prologue work items, each with its partial-sum slot (the matrix's items
@@ -167,6 +179,16 @@ int prologue_grid(int n_items, size_t pro_smem) {
   return std::max(1, std::min(n_items, sms * std::max(per_sm, 1)));
 }
 
+// Dynamic shared memory of the one-pass prologue: the staging buffer of its
+// largest transposed item (0 when no one-pass matrix is transposed).
+size_t one_pass_smem(const Geom* geom, int n_mats) {
+  size_t tb = 0;
+  for (int i = 0; i < n_mats; ++i)
+    if (pro_one_pass(geom[i].cols))
+      tb = std::max(tb, pro_trans_bytes(geom[i].rows, geom[i].cols));
+  return tb;
+}
+
 struct TimingSlot {
   cudaEvent_t ev[kMaxLaunchesPerStep + 1];
   int kind[kMaxLaunchesPerStep];
@@ -193,6 +215,7 @@ struct muon_plan {
   size_t counter_bytes = 0;
   size_t pro_smem = 0;
   int n_one = 0;       // one-pass prologue items (listed first)
+  size_t pro_smem_one = 0;    // dynamic shared memory of the one-pass prologue
   int pro_grid[2] = {0, 0};   // blocks of the one-pass and two-pass prologues
   int max_clusters = 0;
 
@@ -274,8 +297,9 @@ struct LaunchTables {
   const SchedItem* sched;
   long long n_sched;
   int32_t* err;
-  size_t pro_smem;
-  int pro_grid[2];    // blocks of the one-pass and two-pass prologues
+  size_t pro_smem;      // two-pass prologue
+  size_t pro_smem_one;  // one-pass prologue
+  int pro_grid[2];      // blocks of the one-pass and two-pass prologues
   int clusters;       // clusters the schedule was built for (all resident)
 };
 
@@ -283,7 +307,7 @@ struct LaunchTables {
 struct StepScratch {
   float* partials;    // one per prologue item
   float* mat_scale;   // one per matrix
-  int32_t* counters;  // [item counters: 2][tickets: n_mats][done: n_mats * K * 3], zeroed per step
+  int32_t* counters;  // [item counters: 2][done: n_mats * K * 3], zeroed per step
   size_t counter_bytes;
   int n_mats;
 };
@@ -360,18 +384,22 @@ bool fill_caller_fields(MatDev& d, const muon_matrix_t& mt) {
   return true;
 }
 
-bool set_kernel_attributes(size_t pro_smem) {
+bool set_kernel_attributes(size_t pro_smem, size_t pro_smem_one) {
   if (cudaFuncSetAttribute(ns_mega_pair_kernel,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kMegaSmemBytes)) != cudaSuccess)
     return false;
-  if (pro_smem > 48 * 1024 &&
-      (cudaFuncSetAttribute(muon_prologue_kernel<true>,
-                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                            static_cast<int>(pro_smem)) != cudaSuccess ||
-       cudaFuncSetAttribute(muon_prologue_kernel<false>,
-                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                            static_cast<int>(pro_smem)) != cudaSuccess))
+  // (set whenever there is dynamic shared memory: static plus dynamic above
+  // 48 KB needs the opt-in even when the dynamic part alone is below it)
+  if (pro_smem > 0 &&
+      cudaFuncSetAttribute(muon_prologue_kernel<false>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(pro_smem)) != cudaSuccess)
+    return false;
+  if (pro_smem_one > 0 &&
+      cudaFuncSetAttribute(muon_prologue_kernel<true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(pro_smem_one)) != cudaSuccess)
     return false;
   return true;
 }
@@ -395,7 +423,7 @@ cudaLaunchConfig_t pair_launch_config(int clusters, cudaStream_t st,
 // Clusters of two that can be resident at once (the persistent schedule
 // relies on every launched cluster being resident); 0 on failure.
 int query_max_clusters() {
-  if (!set_kernel_attributes(0)) {
+  if (!set_kernel_attributes(0, 0)) {
     cudaGetLastError();
     return 0;
   }
@@ -423,18 +451,18 @@ void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
   HyperDev hd{h.momentum, h.lr, h.weight_decay, h.eps_row, h.eps_frob,
               h.nesterov, h.eq_r};
   int32_t* item_ctr = sc.counters;
-  int32_t* tickets = sc.counters + 2;
-  int32_t* done = sc.counters + 2 + sc.n_mats;
+  int32_t* done = sc.counters + 2;
   cudaMemsetAsync(sc.counters, 0, sc.counter_bytes, st);
   if (t.n_one > 0)
     muon_prologue_kernel<true><<<static_cast<unsigned>(t.pro_grid[0]), kProThreads,
-                                 t.pro_smem, st>>>(
-        t.mats, t.items, t.n_one, hd, sc.partials, tickets, item_ctr, sc.mat_scale);
+                                 t.pro_smem_one, st>>>(t.mats, t.items, t.n_one, hd,
+                                                       sc.partials, item_ctr);
   if (t.n_items > t.n_one)
     muon_prologue_kernel<false><<<static_cast<unsigned>(t.pro_grid[1]), kProThreads,
                                   t.pro_smem, st>>>(
-        t.mats, t.items + t.n_one, t.n_items - t.n_one, hd, sc.partials, tickets,
-        item_ctr + 1, sc.mat_scale);
+        t.mats, t.items + t.n_one, t.n_items - t.n_one, hd, sc.partials, item_ctr + 1);
+  muon_frob_scale_kernel<<<static_cast<unsigned>((sc.n_mats + 7) / 8), 256, 0, st>>>(
+      t.mats, sc.n_mats, sc.partials, h.eps_frob, sc.mat_scale);
   if (rec) rec->after(MUON_KIND_PROLOGUE);
 
   if (ns_steps == 0) {
@@ -488,9 +516,16 @@ const char* muon_status_string(muon_status_t s) {
 }
 
 int32_t muon_step_launches(int32_t ns_steps) {
-  // prologue, then one Newton-Schulz launch for all steps (or the 0-step
-  // finisher); the counter reset is a memset, not a kernel
-  return ns_steps < 0 ? 0 : 2;
+  // one prologue kernel, the Frobenius scale kernel, then one Newton-Schulz
+  // launch for all steps (or the 0-step finisher); the counter reset is a
+  // memset, not a kernel
+  return ns_steps < 0 ? 0 : 3;
+}
+
+int32_t muon_plan_step_launches(const muon_plan_t* plan, int32_t ns_steps) {
+  if (!plan || ns_steps < 0) return 0;
+  const int n_items = static_cast<int>(plan->items.size());
+  return (plan->n_one > 0 ? 1 : 0) + (n_items > plan->n_one ? 1 : 0) + 2;
 }
 
 int32_t ema_update_launches(int32_t n_tensors) {
@@ -530,7 +565,7 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
       plan->items.push_back(ProItem{i, r0, std::min(rt, g.rows - r0),
                                     static_cast<int32_t>(plan->items.size())});
     g.part_count = static_cast<int>(plan->items.size()) - g.part_first;
-    if (g.transposed)
+    if (g.transposed && !pro_one_pass(g.cols))
       plan->pro_smem = std::max(plan->pro_smem,
                                 static_cast<size_t>(rt) * (g.cols + 2) * 2);
     fill_sched_matrix(plan->smats[i], g);
@@ -573,8 +608,10 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
   const size_t err_off = t_off;
   t_off += 256;
   const int n_two = static_cast<int>(plan->items.size()) - plan->n_one;
-  if (plan->max_clusters <= 0 || !set_kernel_attributes(plan->pro_smem) ||
-      (plan->pro_grid[0] = prologue_grid<true>(plan->n_one, plan->pro_smem)) < 0 ||
+  plan->pro_smem_one = one_pass_smem(plan->geom.data(), n_mats);
+  if (plan->max_clusters <= 0 ||
+      !set_kernel_attributes(plan->pro_smem, plan->pro_smem_one) ||
+      (plan->pro_grid[0] = prologue_grid<true>(plan->n_one, plan->pro_smem_one)) < 0 ||
       (plan->pro_grid[1] = prologue_grid<false>(n_two, plan->pro_smem)) < 0 ||
       cudaMalloc(&plan->d_block, t_off) != cudaSuccess) {
     cudaGetLastError();
@@ -742,7 +779,8 @@ muon_status_t muon_step_batched(muon_plan_t* plan, const muon_matrix_t* mats,
   // ---- launches
   LaunchTables t{plan->d_mats, plan->d_items, static_cast<int>(plan->items.size()),
                  plan->n_one, plan->d_sched, plan->sched_len, plan->d_err, plan->pro_smem,
-                 {plan->pro_grid[0], plan->pro_grid[1]}, plan->max_clusters};
+                 plan->pro_smem_one, {plan->pro_grid[0], plan->pro_grid[1]},
+                 plan->max_clusters};
   StepScratch sc{reinterpret_cast<float*>(ws + plan->part_off),
                  reinterpret_cast<float*>(ws + plan->scale_off),
                  reinterpret_cast<int32_t*>(ws + plan->counter_off),
@@ -880,7 +918,7 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
       ++n_items;
     }
     g.part_count = n_items - g.part_first;
-    if (g.transposed)
+    if (g.transposed && !pro_one_pass(g.cols))
       pro_smem = std::max(pro_smem, static_cast<size_t>(rt) * (g.cols + 2) * 2);
     fill_sched_matrix(g_na_smats[i], g);
   }
@@ -931,11 +969,12 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
   const size_t ws_off = t_off;
   if (ws_off + ws_bytes > MUON_NOALLOC_SCRATCH_BYTES) return MUON_ERR_WORKSPACE;
 
-  if (!set_kernel_attributes(pro_smem)) {
+  const size_t pro_smem_one = one_pass_smem(g_na_geom, n_mats);
+  if (!set_kernel_attributes(pro_smem, pro_smem_one)) {
     cudaGetLastError();
     return MUON_ERR_CUDA;
   }
-  const int pro_grid_one = prologue_grid<true>(n_one, pro_smem);
+  const int pro_grid_one = prologue_grid<true>(n_one, pro_smem_one);
   const int pro_grid_two = prologue_grid<false>(n_items - n_one, pro_smem);
   if (pro_grid_one < 0 || pro_grid_two < 0) return MUON_ERR_CUDA;
   char* base = static_cast<char*>(g_noalloc_dev_ptr[dev]);
@@ -964,8 +1003,8 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
   LaunchTables t{reinterpret_cast<const MatDev*>(base + mats_off),
                  reinterpret_cast<const ProItem*>(base + items_off), n_items, n_one,
                  reinterpret_cast<const SchedItem*>(base + sched_off), n_sched,
-                 reinterpret_cast<int32_t*>(base), pro_smem, {pro_grid_one, pro_grid_two},
-                 clusters};
+                 reinterpret_cast<int32_t*>(base), pro_smem, pro_smem_one,
+                 {pro_grid_one, pro_grid_two}, clusters};
   StepScratch sc{reinterpret_cast<float*>(ws + part_off),
                  reinterpret_cast<float*>(ws + scale_off),
                  reinterpret_cast<int32_t*>(ws + counter_off), counter_bytes, n_mats};

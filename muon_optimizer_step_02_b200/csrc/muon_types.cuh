@@ -21,6 +21,15 @@ __host__ __device__ constexpr bool pro_one_pass(int cols) {
   return (cols & 7) == 0 && cols <= kProOneWarps * 1024;
 }
 
+// One-pass prologue: a row of up to 1024 elements per warp, longer rows
+// over wpr = 2, 4 or 8 warps (1024 elements each).
+__host__ __device__ constexpr int pro_warps_per_row(int cols) {
+  return cols <= 1024 ? 1 : cols <= 2048 ? 2 : cols <= 4096 ? 4 : 8;
+}
+// One staging buffer of a transposed one-pass item (32 rows of up to 1024
+// elements, 16 of up to 2048).
+constexpr int kProTransBufCap = 65 * 1024;
+
 // Per-matrix record.  Tensor maps first (64-byte aligned), pointers after.
 struct alignas(64) MatDev {
   CUtensorMap tm_xk[2];  // X ping/pong as a K-major operand, box 64 x 128

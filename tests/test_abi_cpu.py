@@ -62,8 +62,9 @@ def test_constants(L):
     assert binding.status_string(0) == "ok"
     assert "timed out" in binding.status_string(-5)
     assert binding.status_string(-99) == "unknown status"
-    assert L.muon_step_launches(5) == 2
-    assert L.muon_step_launches(0) == 2
+    assert L.muon_step_launches(5) == 3
+    assert L.muon_step_launches(0) == 3
+    assert L.muon_plan_step_launches(None, 5) == 0
     assert L.ema_update_launches(278) == 1
     assert L.ema_update_launches(321) == 2
     assert L.ema_update_launches(0) == 0
