@@ -65,6 +65,11 @@ __all__ = [
     "muon_step_batched",
     "ema_update",
     "ema_update_batched",
+    "linear_ramp",
+    "scheduled_hyper",
+    "AdamWHyper",
+    "adamw_update",
+    "adamw_ema",
     "ns_flops",
 ]
 
@@ -251,6 +256,77 @@ def ema_update(E: np.ndarray, P: np.ndarray, decay: float) -> np.ndarray:
 def ema_update_batched(Es, Ps, decay: float):
     """EMA over every parameter tensor of the model."""
     return [ema_update(E, P, decay) for E, P in zip(Es, Ps)]
+
+
+def linear_ramp(v0: float, v1: float, t0: int, t1: int, t: int) -> float:
+    """A hyper-parameter that moves linearly from v0 at step t0 to v1 at step
+    t1 and holds its end values outside [t0, t1] (t1 <= t0: v0 before t1,
+    v1 from t1 on).
+
+    Pages: PR #1893 table "Architecture and training stack", row "Optimizer":
+    Muon momentum 0.99 "warmup from 0.92 over 1500 steps".  The page gives the
+    end points and the length, not the shape; the straight line between them
+    is taken, with step t (0-based, the number of steps already taken) using
+    the value at t, so the first step uses 0.92 and step 1500 on uses 0.99.
+    """
+    if t1 <= t0:
+        return float(v1 if t >= t1 else v0)
+    f = min(max((t - t0) / (t1 - t0), 0.0), 1.0)
+    return float(v0 + (v1 - v0) * f)
+
+
+def scheduled_hyper(hyper: MuonHyper, mu_ramp, lr_ramp, t: int) -> MuonHyper:
+    """The Muon hyper-parameters of step t when momentum and learning rate
+    follow ramps (each a (v0, v1, t0, t1) tuple, see linear_ramp)."""
+    from dataclasses import replace
+    return replace(hyper, momentum=linear_ramp(*mu_ramp, t),
+                   lr=linear_ramp(*lr_ramp, t))
+
+
+@dataclass(frozen=True)
+class AdamWHyper:
+    """AdamW settings for the non-matrix parameters (embeddings, vectors,
+    scalars).  The pages name the optimizer (PR #1893 table "Architecture and
+    training stack", row "Optimizer": "AdamW on embeddings/scalars") but give
+    none of its settings; these are inputs (the defaults are the commonly
+    published AdamW defaults, not values from the pages)."""
+
+    lr: float = 1e-3
+    beta1: float = 0.9
+    beta2: float = 0.999
+    eps: float = 1e-8
+    weight_decay: float = 0.01
+
+
+def adamw_update(P, G, M, V, h: AdamWHyper, t: int):
+    """One AdamW step (Loshchilov & Hutter's decoupled weight decay with
+    Adam's bias-corrected moments), t = 1 for the first step:
+
+      M' = b1 M + (1 - b1) G
+      V' = b2 V + (1 - b2) G^2
+      P' = P (1 - lr wd) - lr (M' / (1 - b1^t)) / (sqrt(V' / (1 - b2^t)) + eps)
+
+    Returns (P', M', V') in fp64."""
+    P = np.asarray(P, dtype=np.float64)
+    G = np.asarray(G, dtype=np.float64)
+    M = np.asarray(M, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    M_new = h.beta1 * M + (1.0 - h.beta1) * G
+    V_new = h.beta2 * V + (1.0 - h.beta2) * G * G
+    m_hat = M_new / (1.0 - h.beta1 ** t)
+    v_hat = V_new / (1.0 - h.beta2 ** t)
+    P_new = P * (1.0 - h.lr * h.weight_decay) - h.lr * m_hat / (np.sqrt(v_hat) + h.eps)
+    return P_new, M_new, V_new
+
+
+def adamw_ema(P, G, M, V, E, h: AdamWHyper, t: int, decay: float):
+    """The AdamW step of a non-matrix tensor followed by the EMA of its
+    updated value (one pass over the tensor on the GPU side).  The EMA
+    follows the optimizer step, so it averages the new parameters (PR #1584
+    section "Summary": batched EMA over all parameters after the step).
+    Returns (P', M', V', E')."""
+    P_new, M_new, V_new = adamw_update(P, G, M, V, h, t)
+    return P_new, M_new, V_new, ema_update(E, P_new, decay)
 
 
 def ns_flops(rows: int, cols: int, steps: int) -> int:

@@ -404,10 +404,141 @@ def pin_exact_tiny(o):
         assert np.allclose(M1, np.array(Mn, dtype=float), rtol=1e-14)
 
 
+# ---------------------------------------------------------------- schedules
+def pin_ramp(o):
+    """Linear ramp: end values at and beyond the ends, the mean at the
+    midpoint, equal increments per step inside, a step function when the
+    ramp has no length; the pages' momentum warm-up (0.92 -> 0.99 over 1500
+    steps) at its first, middle and last steps."""
+    r = o.linear_ramp
+    assert r(0.92, 0.99, 0, 1500, 0) == 0.92
+    assert abs(r(0.92, 0.99, 0, 1500, 750) - 0.955) < 1e-15
+    assert r(0.92, 0.99, 0, 1500, 1500) == 0.99
+    assert r(0.92, 0.99, 0, 1500, 10 ** 6) == 0.99
+    assert r(0.5, 1.5, 10, 20, 3) == 0.5          # before the start
+    vals = [r(0.5, 1.5, 10, 20, t) for t in range(10, 21)]
+    assert np.allclose(np.diff(vals), 0.1, rtol=0, atol=1e-15)
+    assert r(2.0, 3.0, 5, 5, 4) == 2.0 and r(2.0, 3.0, 5, 5, 5) == 3.0
+    h = o.scheduled_hyper(o.MuonHyper(momentum=0.5, lr=9.0),
+                          (0.92, 0.99, 0, 1500), (0.02, 0.01, 100, 200), 150)
+    assert abs(h.momentum - (0.92 + 0.07 * 0.1)) < 1e-15
+    assert abs(h.lr - 0.015) < 1e-15
+
+
+def pin_ramp_momentum_exact(o):
+    """Momentum under a ramped mu, checked in exact rational arithmetic:
+    with constant G and M_0 = 0, M_T = G * sum_s prod_{k=s+1..T} mu_k where
+    step k (1-based) uses mu at ramp step k - 1."""
+    v0, v1, t0, t1 = Fraction(1, 2), Fraction(7, 8), 0, 3
+    def mu_exact(t):
+        if t >= t1:
+            return v1
+        return v0 + (v1 - v0) * Fraction(t - t0, t1 - t0)
+    G = Fraction(3, 1)
+    T = 5
+    expect = sum(G * np.prod([mu_exact(k - 1) for k in range(s + 1, T + 1)] or [1])
+                 for s in range(1, T + 1))
+    M = np.zeros(1)
+    for t in range(T):
+        mu = o.linear_ramp(float(v0), float(v1), t0, t1, t)
+        assert abs(mu - float(mu_exact(t))) < 1e-15
+        M, _ = o.nesterov_momentum(M, np.array([float(G)]), mu, True)
+    assert abs(M[0] - float(expect)) < 1e-12
+
+
+# ---------------------------------------------------------------- AdamW
+def _adamw_h(o, **kw):
+    base = dict(lr=0.01, beta1=0.9, beta2=0.99, eps=0.0, weight_decay=0.1)
+    base.update(kw)
+    return o.AdamWHyper(**base)
+
+
+def pin_adamw_first_and_constant_steps(o):
+    """From zero moments with eps = 0 the bias-corrected moments of a
+    constant gradient are g and g^2 at every step, so each step moves every
+    entry by lr * sign(g) after the decoupled decay:
+    P_T = P_0 c^T - lr sign(g) (1 + c + ... + c^(T-1)),  c = 1 - lr wd."""
+    rng = np.random.default_rng(20)
+    P0 = rng.standard_normal(9)
+    g = rng.standard_normal(9)
+    h = _adamw_h(o)
+    c = 1 - h.lr * h.weight_decay
+    P, M, V = P0.copy(), np.zeros(9), np.zeros(9)
+    for T in range(1, 12):
+        P, M, V = o.adamw_update(P, g, M, V, h, T)
+        geo = sum(c ** k for k in range(T))
+        assert np.allclose(P, P0 * c ** T - h.lr * np.sign(g) * geo,
+                           rtol=1e-12, atol=1e-14)
+        assert np.allclose(M, g * (1 - h.beta1 ** T), rtol=1e-12)
+        assert np.allclose(V, g * g * (1 - h.beta2 ** T), rtol=1e-12)
+
+
+def pin_adamw_exact_two_steps(o):
+    """Two AdamW steps in exact rational arithmetic with b1 = 1/2, b2 = 1/2
+    and gradients (5, 1): the bias-corrected second moment of step 2 is
+    (b2 g1^2 + g2^2) / (1 + b2) = 9, a perfect square, so the whole update is
+    rational."""
+    F = Fraction
+    b1, b2, lr, wd = F(1, 2), F(1, 2), F(1, 10), F(1, 5)
+    g1, g2, p0 = F(5), F(1), F(3)
+    m1 = (1 - b1) * g1
+    v1 = (1 - b2) * g1 * g1
+    p1 = p0 * (1 - lr * wd) - lr * (m1 / (1 - b1)) / F(5)     # sqrt(v1/(1-b2)) = 5
+    m2 = b1 * m1 + (1 - b1) * g2
+    v2 = b2 * v1 + (1 - b2) * g2 * g2
+    assert v2 / (1 - b2 ** 2) == 9
+    p2 = p1 * (1 - lr * wd) - lr * (m2 / (1 - b1 ** 2)) / F(3)
+    h = o.AdamWHyper(lr=0.1, beta1=0.5, beta2=0.5, eps=0.0, weight_decay=0.2)
+    P, M, V = o.adamw_update(np.array([3.0]), np.array([5.0]), np.zeros(1),
+                             np.zeros(1), h, 1)
+    assert abs(P[0] - float(p1)) < 1e-15
+    P, M, V = o.adamw_update(P, np.array([1.0]), M, V, h, 2)
+    assert abs(P[0] - float(p2)) < 1e-15 and abs(M[0] - float(m2)) < 1e-15
+    assert abs(V[0] - float(v2)) < 1e-15
+
+
+def pin_adamw_invariances(o):
+    """With eps = 0 the AdamW direction is unchanged by a positive rescaling
+    of every gradient and flips with their sign; with lr = 0 nothing moves
+    but the moments."""
+    rng = np.random.default_rng(21)
+    P = rng.standard_normal(6)
+    G1, G2 = rng.standard_normal(6), rng.standard_normal(6)
+    h = _adamw_h(o)
+    def run(s):
+        p, m, v = P.copy(), np.zeros(6), np.zeros(6)
+        p, m, v = o.adamw_update(p, s * G1, m, v, h, 1)
+        p, m, v = o.adamw_update(p, s * G2, m, v, h, 2)
+        return p
+    base = run(1.0)
+    assert np.allclose(run(37.5), base, rtol=1e-12)
+    c2 = (1 - h.lr * h.weight_decay) ** 2
+    assert np.allclose(run(-1.0) - P * c2, -(base - P * c2), rtol=1e-12)
+    p, _, _ = o.adamw_update(P, G1, np.zeros(6), np.zeros(6),
+                             _adamw_h(o, lr=0.0), 1)
+    assert np.array_equal(p, P)
+
+
+def pin_adamw_ema(o):
+    """The fused pass: the EMA averages the updated parameters,
+    E' = d E + (1 - d) P' (checked against the AdamW closed form of a first
+    step, P' = P c - lr sign(g))."""
+    rng = np.random.default_rng(22)
+    P, G, E = rng.standard_normal(5), rng.standard_normal(5), rng.standard_normal(5)
+    h = _adamw_h(o)
+    d = 0.9965
+    P1, M1, V1, E1 = o.adamw_ema(P, G, np.zeros(5), np.zeros(5), E, h, 1, d)
+    Pc = P * (1 - h.lr * h.weight_decay) - h.lr * np.sign(G)
+    assert np.allclose(P1, Pc, rtol=1e-12, atol=1e-15)
+    assert np.allclose(E1, d * E + (1 - d) * Pc, rtol=1e-12, atol=1e-15)
+
+
 ALL_PINS = [
     pin_momentum_closed_form, pin_eq_r_row_norms, pin_frobenius,
     pin_ns_diagonal, pin_ns_conjugated, pin_ns_row_vector, pin_ns_band,
     pin_ns_polar_factor, pin_ns_equivariance, pin_update_zero_grad,
     pin_end_to_end_diagonal, pin_step_row_norms, pin_ema_closed_form,
-    pin_exact_tiny,
+    pin_exact_tiny, pin_ramp, pin_ramp_momentum_exact,
+    pin_adamw_first_and_constant_steps, pin_adamw_exact_two_steps,
+    pin_adamw_invariances, pin_adamw_ema,
 ]

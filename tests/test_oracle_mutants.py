@@ -129,6 +129,56 @@ def _step_eq_r_after_transpose(W, M, G, hyper, coeffs, scale,
         M_new, O
 
 
+def _ramp_off_by_one(v0, v1, t0, t1, t):
+    return mo.__dict__["_orig_ramp"](v0, v1, t0, t1, t + 1)
+
+
+def _ramp_unclamped(v0, v1, t0, t1, t):
+    if t1 <= t0:
+        return float(v1 if t >= t1 else v0)
+    return float(v0 + (v1 - v0) * (t - t0) / (t1 - t0))
+
+
+def _adamw_no_bias_correction(P, G, M, V, h, t):
+    M2 = h.beta1 * np.asarray(M, float) + (1 - h.beta1) * np.asarray(G, float)
+    V2 = h.beta2 * np.asarray(V, float) + (1 - h.beta2) * np.asarray(G, float) ** 2
+    return (np.asarray(P, float) * (1 - h.lr * h.weight_decay)
+            - h.lr * M2 / (np.sqrt(V2) + h.eps), M2, V2)
+
+
+def _adamw_l2(P, G, M, V, h, t):
+    # weight decay folded into the gradient (Adam + L2) instead of decoupled
+    G = np.asarray(G, float) + h.weight_decay * np.asarray(P, float)
+    M2 = h.beta1 * np.asarray(M, float) + (1 - h.beta1) * G
+    V2 = h.beta2 * np.asarray(V, float) + (1 - h.beta2) * G * G
+    mh, vh = M2 / (1 - h.beta1 ** t), V2 / (1 - h.beta2 ** t)
+    return np.asarray(P, float) - h.lr * mh / (np.sqrt(vh) + h.eps), M2, V2
+
+
+def _adamw_swapped_betas(P, G, M, V, h, t):
+    from dataclasses import replace
+    return mo.__dict__["_orig_adamw"](P, G, M, V,
+                                      replace(h, beta1=h.beta2, beta2=h.beta1), t)
+
+
+def _adamw_step_zero_based(P, G, M, V, h, t):
+    return mo.__dict__["_orig_adamw"](P, G, M, V, h, t + 1)
+
+
+def _adamw_abs_second_moment(P, G, M, V, h, t):
+    G = np.asarray(G, float)
+    M2 = h.beta1 * np.asarray(M, float) + (1 - h.beta1) * G
+    V2 = h.beta2 * np.asarray(V, float) + (1 - h.beta2) * np.abs(G)
+    mh, vh = M2 / (1 - h.beta1 ** t), V2 / (1 - h.beta2 ** t)
+    return (np.asarray(P, float) * (1 - h.lr * h.weight_decay)
+            - h.lr * mh / (np.sqrt(vh) + h.eps), M2, V2)
+
+
+def _adamw_ema_old_params(P, G, M, V, E, h, t, decay):
+    P2, M2, V2 = mo.adamw_update(P, G, M, V, h, t)
+    return P2, M2, V2, mo.ema_update(E, P, decay)
+
+
 MUTANTS = {
     "ns_drop_c": ("newton_schulz", _ns_drop_c),
     "ns_gram_wrong_side": ("newton_schulz", _ns_gram_wrong_side),
@@ -148,6 +198,14 @@ MUTANTS = {
     "ema_swapped": ("ema_update", _ema_swapped),
     "step_no_back_transpose": ("muon_step", _step_no_back_transpose),
     "step_eq_r_after_transpose": ("muon_step", _step_eq_r_after_transpose),
+    "ramp_off_by_one": ("linear_ramp", _ramp_off_by_one),
+    "ramp_unclamped": ("linear_ramp", _ramp_unclamped),
+    "adamw_no_bias_correction": ("adamw_update", _adamw_no_bias_correction),
+    "adamw_l2": ("adamw_update", _adamw_l2),
+    "adamw_swapped_betas": ("adamw_update", _adamw_swapped_betas),
+    "adamw_step_zero_based": ("adamw_update", _adamw_step_zero_based),
+    "adamw_abs_second_moment": ("adamw_update", _adamw_abs_second_moment),
+    "adamw_ema_old_params": ("adamw_ema", _adamw_ema_old_params),
 }
 
 
@@ -155,6 +213,8 @@ MUTANTS = {
 def test_mutant_is_caught(name, monkeypatch):
     attr, fn = MUTANTS[name]
     monkeypatch.setitem(mo.__dict__, "_orig_ns", mo.newton_schulz)
+    monkeypatch.setitem(mo.__dict__, "_orig_ramp", mo.linear_ramp)
+    monkeypatch.setitem(mo.__dict__, "_orig_adamw", mo.adamw_update)
     monkeypatch.setattr(mo, attr, fn)
     failed = []
     for pin in pins.ALL_PINS:
