@@ -274,6 +274,11 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         ema_ms = e0.elapsed_time(e1) / reps
 
+    # ---- the fused AdamW + EMA pass over the model's non-matrix parameters
+    # (embeddings, vectors, scalars), each launch timed alone after an L2
+    # flush (its 0.23 GB of traffic is about the size of L2)
+    adamw = adamw_ema_measure(w, stream, max(3, min(args.steps, 20)))
+
     # ---- end to end through the public API with host buffers: pinned
     # gradients copied in every step, the status word read back every step.
     G_pin = [g.pin_memory() for g in rep.G_host]
@@ -364,7 +369,50 @@ def run_ours(args, rank, world, local_rank):
                 "ms": round(ema_ms, 4) if ema_ms else None},
         "breakdown": breakdown,
     }
+    if adamw is not None:
+        a_ms, a_params = adamw
+        a_gbs = 36 * a_params / (a_ms / 1e3) / 1e9
+        line["adamw_ema"] = {"params": a_params, "ms": round(a_ms, 4),
+                             "gbs": round(a_gbs, 1),
+                             "frac": round(a_gbs / peaks["hbm_gbs"], 4),
+                             "bytes_per_param": 36}
     return line
+
+
+def adamw_ema_measure(w, stream, reps):
+    """Device time of one adamw_ema_batched launch over the non-matrix
+    parameters of the 11L x 512d model (None for other workloads)."""
+    import torch
+    from muon_optimizer_step_02_b200 import binding as B
+    if w.ema_decay is None or w.n_mats != 66:
+        return None
+    numels, _ = wl.gpt11_ema_extras()
+    P, G, M, V, E = [], [], [], [], []
+    for i, n in enumerate(numels):
+        p, m, v, e = wl.adamw_state(n, i)
+        P.append(torch.from_numpy(p).cuda())
+        M.append(torch.from_numpy(m).cuda())
+        V.append(torch.from_numpy(v).cuda())
+        E.append(torch.from_numpy(e).cuda())
+        G.append(torch.from_numpy(wl.adamw_grad(n, i, 1)).cuda())
+    hyp = type("AdamW", (), dict(lr=1e-3, beta1=0.9, beta2=0.95, eps=1e-8,
+                                 weight_decay=0.0))
+    run = B.adamw_ema_bind(P, G, M, V, E, hyp, w.ema_decay)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    for t in range(1, 4):
+        run(step_now=t)
+    total = 0.0
+    for t in range(reps):
+        flush.zero_()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        run(step_now=4 + t)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        total += a0.elapsed_time(a1)
+    del flush
+    return total / reps, sum(numels)
 
 
 # --------------------------------------------------------------------------

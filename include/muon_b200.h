@@ -123,6 +123,44 @@ muon_status_t muon_step_batched(muon_plan_t *plan, const muon_matrix_t *mats,
                                 void *workspace, size_t workspace_bytes,
                                 muon_stream_t stream);
 
+/* A hyper-parameter that moves linearly from v0 at step t0 to v1 at step t1
+ * and holds its end values outside [t0, t1] (t1 <= t0: v0 before t1, v1 from
+ * t1 on).  Source: PR #1893 "Record: L_ParallelResiduals_UNetSkips_DepthRecur
+ * _Muon_ 1.0901", table "Architecture and training stack", row "Optimizer":
+ * Muon momentum 0.99 with a warm-up from 0.92 over 1500 steps, i.e.
+ * {0.92, 0.99, 0, 1500}; the page gives the end points and the length, the
+ * straight line between them is this library's reading. */
+typedef struct {
+  float v0;
+  float v1;
+  int32_t t0;
+  int32_t t1;
+} muon_ramp_t;
+
+/* Momentum and learning rate of a scheduled step (both finite ramps; the
+ * momentum ramp stays in [0, 1)). */
+typedef struct {
+  muon_ramp_t momentum;
+  muon_ramp_t lr;
+} muon_schedule_t;
+
+/* muon_step_batched with the momentum and the learning rate taken on the
+ * device from `sched` at the step number *step_dev (device int32, owned by
+ * the caller, 4-byte aligned, 0 before the first step); the call advances
+ * *step_dev by one on the device.  hyper->momentum and hyper->lr are
+ * ignored.  Because nothing of the step number passes through the host, a
+ * CUDA graph captured from one call (after one uncaptured call with the same
+ * buffers and step count, see muon_step_batched) replays every later step
+ * with the right schedule values.  Errors as muon_step_batched, plus
+ * MUON_ERR_INVALID_ARG for a missing or non-finite schedule or step_dev, and
+ * MUON_ERR_ALIGNMENT for a misaligned step_dev. */
+muon_status_t muon_step_batched_sched(muon_plan_t *plan, const muon_matrix_t *mats,
+                                      const muon_hyper_t *hyper,
+                                      const muon_schedule_t *sched, int32_t *step_dev,
+                                      const float *ns_coeffs, int32_t ns_steps,
+                                      void *workspace, size_t workspace_bytes,
+                                      muon_stream_t stream);
+
 /* E' = decay E + (1 - decay) P for n_tensors tensors in one pass.
  *  ema     host array of device fp32 pointers (updated in place).
  *  params  host array of device fp32 pointers (read only).
@@ -132,6 +170,50 @@ muon_status_t muon_step_batched(muon_plan_t *plan, const muon_matrix_t *mats,
 muon_status_t ema_update_batched(float *const *ema, const float *const *params,
                                  const int64_t *numel, int32_t n_tensors,
                                  float decay, muon_stream_t stream);
+
+/* AdamW settings of the non-matrix parameters.  Source: PR #1893 "Record:
+ * L_ParallelResiduals_UNetSkips_DepthRecur_Muon_ 1.0901", table
+ * "Architecture and training stack", row "Optimizer": AdamW on embeddings
+ * and scalars (the page gives no setting; all are inputs).  lr, weight_decay
+ * finite; beta1, beta2 in [0, 1); eps >= 0. */
+typedef struct {
+  float lr;
+  float beta1;
+  float beta2;
+  float eps;
+  float weight_decay;
+} adamw_hyper_t;
+
+/* One non-matrix tensor: device fp32 arrays of numel elements (numel >= 0).
+ * param, exp_avg (first moment) and exp_avg_sq (second moment) are updated
+ * in place, grad is read, ema (may be NULL: no EMA for this tensor) is
+ * updated in place.  4-byte alignment required; when all five are 16-byte
+ * aligned the tensor takes the vectorised path.  Arrays must not overlap. */
+typedef struct {
+  float *param;
+  const float *grad;
+  float *exp_avg;
+  float *exp_avg_sq;
+  float *ema;
+  int64_t numel;
+} adamw_tensor_t;
+
+/* AdamW step of every tensor, then the EMA of the updated parameter, in one
+ * pass over memory (the other optimizer of the training step, fused into the
+ * EMA sweep):
+ *   m' = b1 m + (1 - b1) g;  v' = b2 v + (1 - b2) g^2;
+ *   p' = p (1 - lr wd) - lr (m' / (1 - b1^t)) / (sqrt(v' / (1 - b2^t)) + eps);
+ *   e' = decay e + (1 - decay) p'.
+ * t is `step` (>= 1) when step_dev is NULL; otherwise t = *step_dev + 1,
+ * *step_dev (device int32, 4-byte aligned) counting the steps already taken,
+ * and the call advances *step_dev by one after its kernels, so that a CUDA
+ * graph captured from one call serves every step.  Use a counter of its own
+ * (muon_step_batched_sched advances its counter too).  Asynchronous on
+ * `stream`; argument errors are returned before anything is enqueued. */
+muon_status_t adamw_ema_batched(const adamw_tensor_t *tensors, int32_t n_tensors,
+                                const adamw_hyper_t *hyper, int32_t step,
+                                int32_t *step_dev, float ema_decay,
+                                muon_stream_t stream);
 
 /* Synchronises `stream`, reads and clears the plan's device error word.
  * Returns MUON_ERR_TIMEOUT if a kernel gave up on a bounded wait since the
@@ -171,6 +253,9 @@ muon_status_t muon_plan_timing_read(muon_plan_t *plan, int32_t *launches,
 int32_t muon_step_launches(int32_t ns_steps);
 int32_t muon_plan_step_launches(const muon_plan_t *plan, int32_t ns_steps);
 int32_t ema_update_launches(int32_t n_tensors);
+/* Launches of adamw_ema_batched (with_step_dev: 1 if a device counter is
+ * advanced). */
+int32_t adamw_ema_launches(int32_t n_tensors, int32_t with_step_dev);
 
 /* Test hook: fault 1 makes the tensor-core kernel's load warp skip one
  * stage of its first tile in block 0, so that the consumer's bounded wait

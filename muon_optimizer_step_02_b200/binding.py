@@ -41,6 +41,32 @@ class muon_hyper_t(Structure):
                 ("eq_r", c_int32)]
 
 
+class muon_ramp_t(Structure):
+    _fields_ = [("v0", c_float), ("v1", c_float), ("t0", c_int32),
+                ("t1", c_int32)]
+
+
+class muon_schedule_t(Structure):
+    _fields_ = [("momentum", muon_ramp_t), ("lr", muon_ramp_t)]
+
+
+def make_schedule(momentum_ramp, lr_ramp) -> muon_schedule_t:
+    """(v0, v1, t0, t1) ramps for the momentum and the learning rate."""
+    m, l = momentum_ramp, lr_ramp
+    return muon_schedule_t(muon_ramp_t(float(m[0]), float(m[1]), int(m[2]), int(m[3])),
+                           muon_ramp_t(float(l[0]), float(l[1]), int(l[2]), int(l[3])))
+
+
+class adamw_hyper_t(Structure):
+    _fields_ = [("lr", c_float), ("beta1", c_float), ("beta2", c_float),
+                ("eps", c_float), ("weight_decay", c_float)]
+
+
+class adamw_tensor_t(Structure):
+    _fields_ = [("param", c_void_p), ("grad", c_void_p), ("exp_avg", c_void_p),
+                ("exp_avg_sq", c_void_p), ("ema", c_void_p), ("numel", c_int64)]
+
+
 class MuonError(RuntimeError):
     def __init__(self, status: int, what: str):
         super().__init__(f"{what}: {status_string(status)} ({status})")
@@ -84,6 +110,18 @@ def lib():
     L.muon_plan_timing_read.argtypes = [c_void_p, POINTER(c_int32),
                                         POINTER(c_double), c_int32]
     L.muon_plan_timing_read.restype = c_int32
+    L.muon_step_batched_sched.argtypes = [c_void_p, POINTER(muon_matrix_t),
+                                          POINTER(muon_hyper_t),
+                                          POINTER(muon_schedule_t), c_void_p,
+                                          POINTER(c_float), c_int32, c_void_p,
+                                          c_size_t, c_void_p]
+    L.muon_step_batched_sched.restype = c_int32
+    L.adamw_ema_batched.argtypes = [POINTER(adamw_tensor_t), c_int32,
+                                    POINTER(adamw_hyper_t), c_int32, c_void_p,
+                                    c_float, c_void_p]
+    L.adamw_ema_batched.restype = c_int32
+    L.adamw_ema_launches.argtypes = [c_int32, c_int32]
+    L.adamw_ema_launches.restype = c_int32
     L.muon_step_launches.argtypes = [c_int32]
     L.muon_step_launches.restype = c_int32
     L.muon_plan_step_launches.argtypes = [c_void_p, c_int32]
@@ -160,20 +198,24 @@ class MuonPlan:
 
     def step(self, weights, momenta, grads, hyper, coeffs, workspace,
              update_scales: Optional[Sequence[float]] = None,
-             update_out=None, stream=None):
-        """One batched Muon step (muon_step_batched).  weights/momenta: fp32
-        CUDA tensors (updated in place); grads: bf16 CUDA tensors; hyper: an
+             update_out=None, stream=None, schedule=None, step_dev=None):
+        """One batched Muon step (muon_step_batched, or with `schedule` and
+        `step_dev` muon_step_batched_sched).  weights/momenta: fp32 CUDA
+        tensors (updated in place); grads: bf16 CUDA tensors; hyper: an
         object with momentum, lr, weight_decay, eps_row, eps_frob, nesterov,
         eq_r; coeffs: ns_steps rows of (a, b, c)."""
         self.bind(weights, momenta, grads, hyper, coeffs, workspace,
-                  update_scales, update_out)(stream)
+                  update_scales, update_out, schedule, step_dev)(stream)
 
     def bind(self, weights, momenta, grads, hyper, coeffs, workspace,
              update_scales: Optional[Sequence[float]] = None,
-             update_out=None):
+             update_out=None, schedule=None, step_dev=None):
         """Checks and marshals the arguments once; returns a callable
-        `run(stream=None)` that enqueues muon_step_batched with them.  The
-        tensors must stay alive and in place while the callable is used."""
+        `run(stream=None)` that enqueues muon_step_batched with them (or
+        muon_step_batched_sched when `schedule`, a pair of (v0, v1, t0, t1)
+        ramps for momentum and lr, and `step_dev`, a one-element int32 CUDA
+        tensor holding the step number, are given).  The tensors must stay
+        alive and in place while the callable is used."""
         import torch
         n = len(self.shapes)
         if not (len(weights) == len(momenta) == len(grads) == n):
@@ -205,10 +247,24 @@ class MuonPlan:
         carr = (c_float * max(len(flat), 1))(*flat)
         _check_tensor(workspace, torch.uint8, (workspace.numel(),),
                       "workspace")
-        fn = lib().muon_step_batched
         h, hp_ref = self._h, ctypes.byref(hp)
         ws_ptr, ws_n = workspace.data_ptr(), workspace.numel()
         keep = (mats, hp, carr, weights, momenta, grads, update_out, workspace)
+        if schedule is not None:
+            if step_dev is None:
+                raise ValueError("a schedule needs step_dev")
+            _check_tensor(step_dev, torch.int32, (1,), "step_dev")
+            sch = make_schedule(*schedule)
+            fn_s = lib().muon_step_batched_sched
+            sch_ref, sp = ctypes.byref(sch), step_dev.data_ptr()
+            keep = keep + (sch, step_dev)
+
+            def run_sched(stream=None):
+                _ = keep
+                _check(fn_s(h, mats, hp_ref, sch_ref, sp, carr, k, ws_ptr, ws_n,
+                            _stream_handle(stream)), "muon_step_batched_sched")
+            return run_sched
+        fn = lib().muon_step_batched
 
         def run(stream=None):
             _ = keep
@@ -297,6 +353,63 @@ def ema_bind(emas: Sequence, params: Sequence, decay: float):
 
 def step_launches(ns_steps: int) -> int:
     return int(lib().muon_step_launches(int(ns_steps)))
+
+
+def adamw_ema_bind(params: Sequence, grads: Sequence, exp_avgs: Sequence,
+                   exp_avg_sqs: Sequence, emas: Sequence, hyper, ema_decay: float,
+                   step: int = 1, step_dev=None):
+    """Marshals adamw_ema_batched once and returns `run(step=None,
+    stream=None)`.  All tensors fp32 CUDA, contiguous, same numel per index;
+    emas[i] may be None.  hyper: an object with lr, beta1, beta2, eps,
+    weight_decay.  With step_dev (one-element int32 CUDA tensor) the device
+    counter gives the step; otherwise `step` (or run's argument)."""
+    import torch
+    n = len(params)
+    if not (len(grads) == len(exp_avgs) == len(exp_avg_sqs) == len(emas) == n):
+        raise ValueError("one grad, exp_avg, exp_avg_sq and ema entry per param")
+    arr = (adamw_tensor_t * max(n, 1))()
+    for i in range(n):
+        k = params[i].numel()
+        for t, what in ((params[i], "params"), (grads[i], "grads"),
+                        (exp_avgs[i], "exp_avgs"), (exp_avg_sqs[i], "exp_avg_sqs")):
+            _check_tensor(t, torch.float32, (t.numel(),) if t.dim() == 1 else tuple(t.shape),
+                          f"{what}[{i}]")
+            if t.numel() != k:
+                raise ValueError(f"{what}[{i}] has {t.numel()} elements, expected {k}")
+        e = emas[i]
+        if e is not None:
+            _check_tensor(e, torch.float32, tuple(e.shape), f"emas[{i}]")
+            if e.numel() != k:
+                raise ValueError(f"emas[{i}] has {e.numel()} elements, expected {k}")
+        arr[i] = adamw_tensor_t(params[i].data_ptr(), grads[i].data_ptr(),
+                                exp_avgs[i].data_ptr(), exp_avg_sqs[i].data_ptr(),
+                                e.data_ptr() if e is not None else None, k)
+    hp = adamw_hyper_t(float(hyper.lr), float(hyper.beta1), float(hyper.beta2),
+                       float(hyper.eps), float(hyper.weight_decay))
+    sp = None
+    if step_dev is not None:
+        _check_tensor(step_dev, torch.int32, (1,), "step_dev")
+        sp = step_dev.data_ptr()
+    fn = lib().adamw_ema_batched
+    keep = (arr, hp, list(params), list(grads), list(exp_avgs), list(exp_avg_sqs),
+            list(emas), step_dev)
+    hp_ref = ctypes.byref(hp)
+
+    def run(step_now: Optional[int] = None, stream=None):
+        _ = keep
+        _check(fn(arr, n, hp_ref, int(step if step_now is None else step_now), sp,
+                  float(ema_decay), _stream_handle(stream)), "adamw_ema_batched")
+    return run
+
+
+def adamw_ema_batched(params, grads, exp_avgs, exp_avg_sqs, emas, hyper,
+                      ema_decay: float, step: int = 1, step_dev=None, stream=None):
+    adamw_ema_bind(params, grads, exp_avgs, exp_avg_sqs, emas, hyper, ema_decay,
+                   step, step_dev)(stream=stream)
+
+
+def adamw_ema_launches(n_tensors: int, with_step_dev: bool = False) -> int:
+    return int(lib().adamw_ema_launches(int(n_tensors), int(bool(with_step_dev))))
 
 
 def ema_launches(n_tensors: int) -> int:

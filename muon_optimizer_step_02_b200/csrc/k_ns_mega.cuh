@@ -62,6 +62,7 @@ struct MegaParams {
   int32_t fault, fresh;
   float a[kMegaMaxSteps], b[kMegaMaxSteps], c[kMegaMaxSteps];
   float lr, wd, eps_frob;
+  const float* lr_dev;    // scheduled learning rate of the step, or null (use lr)
 };
 
 // Shared memory: the operand ring (per stage 16 KB of A rows + 16 KB of B
@@ -595,8 +596,9 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
         // W <- W (1 - lr wd) - lr scale O over this warp's four blocks; the
         // next block's W is already in registers (loaded two blocks ahead,
         // the first two before the accumulator was ready).
-        const float decay = 1.f - p.lr * p.wd;
-        const float step = p.lr * md->update_scale;
+        const float lr = p.lr_dev ? *p.lr_dev : p.lr;
+        const float decay = 1.f - lr * p.wd;
+        const float step = lr * md->update_scale;
         auto block = [&](int j, float (&wv)[32]) {
           float v[32];
           tmem_load_32cols(tbase + (half + 2 * j) * 32, v);

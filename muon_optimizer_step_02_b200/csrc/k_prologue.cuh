@@ -194,7 +194,7 @@ muon_prologue_kernel(const MatDev* __restrict__ mats,
     const int sld = cols + 2;  // staging row stride (elements)
     __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(pro_smem);
     const int nch = (cols + 255) / 256;
-    const float mu = h.mu;
+    const float mu = h.step ? linear_ramp(h.mu_v0, h.mu_v1, h.mu_t0, h.mu_t1, *h.step) : h.mu;
 
     float fro = 0.f;
     if constexpr (kOnePass) {
@@ -387,10 +387,19 @@ muon_prologue_kernel(const MatDev* __restrict__ mats,
 // The Frobenius scale s = 1 / (||X~||_F + eps_frob) of every matrix from its
 // prologue partials: one warp per matrix, lane l adds slots l, l + 32, ...
 // and the warp's butterfly adds the lanes, the same order on every run.
+//
+// With a schedule, thread 0 of block 0 also resolves the step's learning
+// rate into *lr_slot and advances the step counter: every prologue block has
+// read the counter by now, and the later kernels of the step read the slot.
 __global__ void __launch_bounds__(256)
 muon_frob_scale_kernel(const MatDev* __restrict__ mats, int n_mats,
-                       const float* __restrict__ partials, float eps_frob,
+                       const float* __restrict__ partials, HyperDev h,
                        float* __restrict__ mat_scale) {
+  if (h.step && blockIdx.x == 0 && threadIdx.x == 0) {
+    const int32_t t = *h.step;
+    *h.lr_slot = linear_ramp(h.lr_v0, h.lr_v1, h.lr_t0, h.lr_t1, t);
+    *h.step = t + 1;
+  }
   const int mat = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (mat >= n_mats) return;
@@ -398,7 +407,7 @@ muon_frob_scale_kernel(const MatDev* __restrict__ mats, int n_mats,
   float s = 0.f;
   for (int i = lane; i < md.part_count; i += 32) s += partials[md.part_first + i];
   s = warp_allreduce_sum(s);
-  if (lane == 0) mat_scale[mat] = 1.f / (sqrtf(s) + eps_frob);
+  if (lane == 0) mat_scale[mat] = 1.f / (sqrtf(s) + h.eps_frob);
 }
 
 // ns_steps == 0: O = s X~ straight from the prologue's output, then the
@@ -406,10 +415,12 @@ muon_frob_scale_kernel(const MatDev* __restrict__ mats, int n_mats,
 __global__ void __launch_bounds__(kProThreads)
 muon_final_noiter_kernel(const MatDev* __restrict__ mats,
                          const ProItem* __restrict__ items,
-                         const float* __restrict__ mat_scale, float lr, float wd) {
+                         const float* __restrict__ mat_scale, float lr_host,
+                         const float* __restrict__ lr_dev, float wd) {
   const ProItem it = items[blockIdx.x];
   const MatDev& md = mats[it.mat];
   const float s = mat_scale[it.mat];
+  const float lr = lr_dev ? *lr_dev : lr_host;
   const float decay = 1.f - lr * wd;
   const float step = lr * md.update_scale;
   const int cols = md.cols;

@@ -22,6 +22,7 @@
 #include "muon_b200.h"
 
 
+#include "k_adamw_ema.cuh"
 #include "k_ema.cuh"
 #include "k_ns_mega.cuh"
 #include "k_prologue.cuh"
@@ -212,6 +213,7 @@ struct muon_plan {
   size_t part_off = 0;
   size_t scale_off = 0;
   size_t counter_off = 0;
+  size_t lr_slot_off = 0;
   size_t counter_bytes = 0;
   size_t pro_smem = 0;
   int n_one = 0;       // one-pass prologue items (listed first)
@@ -310,6 +312,7 @@ struct StepScratch {
   int32_t* counters;  // [item counters: 2][done: n_mats * K * 3], zeroed per step
   size_t counter_bytes;
   int n_mats;
+  float* lr_slot;     // the scheduled learning rate of the step (or null)
 };
 
 muon_status_t validate_hyper(const muon_hyper_t* hyper, const float* ns_coeffs,
@@ -446,10 +449,31 @@ void fill_sched_matrix(SchedMatrix& s, const Geom& g) {
 
 // counter reset -> prologue -> Newton-Schulz (or finisher for 0 steps).
 void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
+                  const muon_schedule_t* sched, int32_t* step_dev,
                   const float* ns_coeffs, int32_t ns_steps, const StepScratch& sc,
                   int fault, bool fresh, cudaStream_t st, Recorder* rec) {
-  HyperDev hd{h.momentum, h.lr, h.weight_decay, h.eps_row, h.eps_frob,
-              h.nesterov, h.eq_r};
+  HyperDev hd{};
+  hd.mu = h.momentum;
+  hd.lr = h.lr;
+  hd.wd = h.weight_decay;
+  hd.eps_row = h.eps_row;
+  hd.eps_frob = h.eps_frob;
+  hd.nesterov = h.nesterov;
+  hd.eq_r = h.eq_r;
+  const float* lr_dev = nullptr;
+  if (sched) {
+    hd.step = step_dev;
+    hd.lr_slot = sc.lr_slot;
+    hd.mu_v0 = sched->momentum.v0;
+    hd.mu_v1 = sched->momentum.v1;
+    hd.mu_t0 = sched->momentum.t0;
+    hd.mu_t1 = sched->momentum.t1;
+    hd.lr_v0 = sched->lr.v0;
+    hd.lr_v1 = sched->lr.v1;
+    hd.lr_t0 = sched->lr.t0;
+    hd.lr_t1 = sched->lr.t1;
+    lr_dev = sc.lr_slot;
+  }
   int32_t* item_ctr = sc.counters;
   int32_t* done = sc.counters + 2;
   cudaMemsetAsync(sc.counters, 0, sc.counter_bytes, st);
@@ -462,12 +486,12 @@ void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
                                   t.pro_smem, st>>>(
         t.mats, t.items + t.n_one, t.n_items - t.n_one, hd, sc.partials, item_ctr + 1);
   muon_frob_scale_kernel<<<static_cast<unsigned>((sc.n_mats + 7) / 8), 256, 0, st>>>(
-      t.mats, sc.n_mats, sc.partials, h.eps_frob, sc.mat_scale);
+      t.mats, sc.n_mats, sc.partials, hd, sc.mat_scale);
   if (rec) rec->after(MUON_KIND_PROLOGUE);
 
   if (ns_steps == 0) {
     muon_final_noiter_kernel<<<static_cast<unsigned>(t.n_items), kProThreads, 0,
-                               st>>>(t.mats, t.items, sc.mat_scale, h.lr,
+                               st>>>(t.mats, t.items, sc.mat_scale, h.lr, lr_dev,
                                      h.weight_decay);
     if (rec) rec->after(MUON_KIND_FINAL);
     return;
@@ -488,6 +512,7 @@ void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
     p.c[k] = ns_coeffs[3 * k + 2];
   }
   p.lr = h.lr;
+  p.lr_dev = lr_dev;
   p.wd = h.weight_decay;
   p.eps_frob = h.eps_frob;
   cudaLaunchAttribute attr[1];
@@ -530,6 +555,11 @@ int32_t muon_plan_step_launches(const muon_plan_t* plan, int32_t ns_steps) {
 
 int32_t ema_update_launches(int32_t n_tensors) {
   return n_tensors <= 0 ? 0 : (n_tensors + kEmaMaxSegs - 1) / kEmaMaxSegs;
+}
+
+int32_t adamw_ema_launches(int32_t n_tensors, int32_t with_step_dev) {
+  if (n_tensors < 0) return 0;
+  return (n_tensors + kAdamMaxSegs - 1) / kAdamMaxSegs + (with_step_dev ? 1 : 0);
 }
 
 muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
@@ -586,6 +616,8 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
   plan->counter_off = off;
   plan->counter_bytes = counter_bytes_for(n_mats, max_ns_steps);
   off = align_up(off + plan->counter_bytes, 1024);
+  plan->lr_slot_off = off;   // the scheduled learning rate of a step
+  off = align_up(off + sizeof(float), 1024);
   plan->ws_bytes = off;
 
   if (cudaGetDevice(&plan->device) != cudaSuccess ||
@@ -709,15 +741,28 @@ muon_status_t muon_get_last_error(muon_plan_t* plan, muon_stream_t stream) {
   return MUON_OK;
 }
 
-muon_status_t muon_step_batched(muon_plan_t* plan, const muon_matrix_t* mats,
-                                const muon_hyper_t* hyper,
-                                const float* ns_coeffs, int32_t ns_steps,
-                                void* workspace, size_t workspace_bytes,
-                                muon_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+bool finite_ramp(const muon_ramp_t& r) { return finite(r.v0) && finite(r.v1); }
+
+// The plain and the scheduled step (sched non-null).
+muon_status_t step_impl(muon_plan_t* plan, const muon_matrix_t* mats,
+                        const muon_hyper_t* hyper, const muon_schedule_t* sched,
+                        int32_t* step_dev, const float* ns_coeffs, int32_t ns_steps,
+                        void* workspace, size_t workspace_bytes, muon_stream_t stream) {
   // ---- validation (host, before anything is enqueued)
   if (!plan || !mats) return MUON_ERR_INVALID_ARG;
   muon_status_t vs = validate_hyper(hyper, ns_coeffs, ns_steps, plan->max_ns);
   if (vs != MUON_OK) return vs;
+  if (sched) {
+    if (!step_dev || !finite_ramp(sched->momentum) || !finite_ramp(sched->lr) ||
+        sched->momentum.v0 < 0.f || sched->momentum.v0 >= 1.f ||
+        sched->momentum.v1 < 0.f || sched->momentum.v1 >= 1.f)
+      return MUON_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(step_dev) & 3u) != 0) return MUON_ERR_ALIGNMENT;
+  }
   if (!workspace || workspace_bytes < plan->ws_bytes) return MUON_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MUON_ERR_WORKSPACE;
   for (int i = 0; i < plan->n_mats; ++i) {
@@ -784,13 +829,38 @@ muon_status_t muon_step_batched(muon_plan_t* plan, const muon_matrix_t* mats,
   StepScratch sc{reinterpret_cast<float*>(ws + plan->part_off),
                  reinterpret_cast<float*>(ws + plan->scale_off),
                  reinterpret_cast<int32_t*>(ws + plan->counter_off),
-                 counter_bytes_for(plan->n_mats, ns_steps), plan->n_mats};
+                 counter_bytes_for(plan->n_mats, ns_steps), plan->n_mats,
+                 reinterpret_cast<float*>(ws + plan->lr_slot_off)};
   Recorder rec(plan, st);
-  enqueue_step(t, *hyper, ns_coeffs, ns_steps, sc, plan->fault, changed, st,
-               plan->timing ? &rec : nullptr);
+  enqueue_step(t, *hyper, sched, step_dev, ns_coeffs, ns_steps, sc, plan->fault, changed,
+               st, plan->timing ? &rec : nullptr);
   rec.finish();
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+muon_status_t muon_step_batched(muon_plan_t* plan, const muon_matrix_t* mats,
+                                const muon_hyper_t* hyper,
+                                const float* ns_coeffs, int32_t ns_steps,
+                                void* workspace, size_t workspace_bytes,
+                                muon_stream_t stream) {
+  return step_impl(plan, mats, hyper, nullptr, nullptr, ns_coeffs, ns_steps, workspace,
+                   workspace_bytes, stream);
+}
+
+muon_status_t muon_step_batched_sched(muon_plan_t* plan, const muon_matrix_t* mats,
+                                      const muon_hyper_t* hyper,
+                                      const muon_schedule_t* sched, int32_t* step_dev,
+                                      const float* ns_coeffs, int32_t ns_steps,
+                                      void* workspace, size_t workspace_bytes,
+                                      muon_stream_t stream) {
+  if (!sched) return MUON_ERR_INVALID_ARG;
+  return step_impl(plan, mats, hyper, sched, step_dev, ns_coeffs, ns_steps, workspace,
+                   workspace_bytes, stream);
 }
 
 muon_status_t ema_update_batched(float* const* ema, const float* const* params,
@@ -836,6 +906,64 @@ muon_status_t ema_update_batched(float* const* ema, const float* const* params,
     const unsigned grid = static_cast<unsigned>(std::min<long long>(want, 8ll * sms));
     ema_update_kernel<<<grid, kEmaThreads, 0, st>>>(p);
   }
+  if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
+  return MUON_OK;
+}
+
+muon_status_t adamw_ema_batched(const adamw_tensor_t* tensors, int32_t n_tensors,
+                                const adamw_hyper_t* hyper, int32_t step,
+                                int32_t* step_dev, float ema_decay, muon_stream_t stream) {
+  if (n_tensors < 0 || !hyper || !finite(ema_decay)) return MUON_ERR_INVALID_ARG;
+  if (n_tensors > 0 && !tensors) return MUON_ERR_INVALID_ARG;
+  const adamw_hyper_t& h = *hyper;
+  if (!finite(h.lr) || !finite(h.weight_decay) || !finite(h.eps) || h.eps < 0.f ||
+      !(h.beta1 >= 0.f && h.beta1 < 1.f) || !(h.beta2 >= 0.f && h.beta2 < 1.f))
+    return MUON_ERR_INVALID_ARG;
+  if (!step_dev && step < 1) return MUON_ERR_INVALID_ARG;
+  if (step_dev && (reinterpret_cast<uintptr_t>(step_dev) & 3u) != 0) return MUON_ERR_ALIGNMENT;
+  for (int i = 0; i < n_tensors; ++i) {
+    const adamw_tensor_t& x = tensors[i];
+    if (x.numel < 0) return MUON_ERR_INVALID_ARG;
+    if (x.numel == 0) continue;
+    if (!x.param || !x.grad || !x.exp_avg || !x.exp_avg_sq) return MUON_ERR_INVALID_ARG;
+    if (((reinterpret_cast<uintptr_t>(x.param) | reinterpret_cast<uintptr_t>(x.grad) |
+          reinterpret_cast<uintptr_t>(x.exp_avg) | reinterpret_cast<uintptr_t>(x.exp_avg_sq) |
+          reinterpret_cast<uintptr_t>(x.ema)) & 3u) != 0)
+      return MUON_ERR_ALIGNMENT;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int sms = 148;
+  {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MUON_ERR_CUDA;
+  }
+  for (int first = 0; first < n_tensors; first += kAdamMaxSegs) {
+    AdamParams a{};
+    a.step_dev = step_dev;
+    a.step = step;
+    a.lr = h.lr;
+    a.b1 = h.beta1;
+    a.b2 = h.beta2;
+    a.eps = h.eps;
+    a.wd = h.weight_decay;
+    a.d = ema_decay;
+    long long units = 0;
+    int ns = 0;
+    for (int i = first; i < std::min(n_tensors, first + kAdamMaxSegs); ++i, ++ns) {
+      const adamw_tensor_t& x = tensors[i];
+      a.seg[ns] = AdamSeg{x.param, x.grad, x.exp_avg, x.exp_avg_sq, x.ema, x.numel, units};
+      units += (x.numel + 3) / 4;
+    }
+    a.n_seg = ns;
+    a.total_units = units;
+    // (launched even when empty, so that the launch count is fixed)
+    const long long want = std::max(1ll, (units + kAdamThreads - 1) / kAdamThreads);
+    const unsigned grid = static_cast<unsigned>(std::min<long long>(want, 8ll * sms));
+    adamw_ema_kernel<<<grid, kAdamThreads, 0, st>>>(a);
+  }
+  if (step_dev) adamw_step_advance_kernel<<<1, 1, 0, st>>>(step_dev);
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
 }
@@ -1007,8 +1135,9 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
                  {pro_grid_one, pro_grid_two}, clusters};
   StepScratch sc{reinterpret_cast<float*>(ws + part_off),
                  reinterpret_cast<float*>(ws + scale_off),
-                 reinterpret_cast<int32_t*>(ws + counter_off), counter_bytes, n_mats};
-  enqueue_step(t, *hyper, ns_coeffs, ns_steps, sc, 0, true, st, nullptr);
+                 reinterpret_cast<int32_t*>(ws + counter_off), counter_bytes, n_mats,
+                 nullptr};
+  enqueue_step(t, *hyper, nullptr, nullptr, ns_coeffs, ns_steps, sc, 0, true, st, nullptr);
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
 }

@@ -88,7 +88,25 @@ struct SchedItem {
 struct HyperDev {
   float mu, lr, wd, eps_row, eps_frob;
   int32_t nesterov, eq_r;
+  // Scheduled momentum and learning rate (when `step` is not null): the
+  // values at step *step of two linear ramps.  The Frobenius scale kernel
+  // writes the step's learning rate to *lr_slot for the Newton-Schulz or
+  // finishing kernel and advances *step.
+  int32_t* step;
+  float* lr_slot;
+  float mu_v0, mu_v1, lr_v0, lr_v1;
+  int32_t mu_t0, mu_t1, lr_t0, lr_t1;
 };
+
+// A value moving linearly from v0 at step t0 to v1 at step t1, holding its
+// end values outside [t0, t1] (t1 <= t0: v0 before t1, v1 from t1 on).
+__host__ __device__ inline float linear_ramp(float v0, float v1, int32_t t0, int32_t t1,
+                                             int32_t t) {
+  if (t1 <= t0) return t >= t1 ? v1 : v0;
+  float f = static_cast<float>(t - t0) / static_cast<float>(t1 - t0);
+  f = f < 0.f ? 0.f : (f > 1.f ? 1.f : f);
+  return v0 + (v1 - v0) * f;
+}
 
 enum NsMode : int32_t { kModeGram = 0, kModePoly = 1, kModeApply = 2 };
 

@@ -179,7 +179,7 @@ def workload(idx: int) -> Workload:
 # Random inputs
 # --------------------------------------------------------------------------
 
-KIND_W, KIND_G, KIND_ROWSCALE, KIND_E, KIND_P = 1, 2, 3, 4, 5
+KIND_W, KIND_G, KIND_ROWSCALE, KIND_E, KIND_P, KIND_ADAM = 1, 2, 3, 4, 5, 6
 
 
 def _rng(seed: int, wid: int, idx: int, step: int, kind: int):
@@ -226,6 +226,24 @@ def ema_pair(w: Workload, idx: int, seed: int = 1337):
     e = _rng(seed, w.wid, idx, 0, KIND_E).standard_normal(n, dtype=np.float32)
     p = _rng(seed, w.wid, idx, 0, KIND_P).standard_normal(n, dtype=np.float32)
     return e * np.float32(0.02), p * np.float32(0.02)
+
+
+def adamw_state(numel: int, idx: int, seed: int = 1337, wid: int = 200):
+    """(P, M, V, E) fp32 arrays for non-matrix tensor idx of an AdamW + EMA
+    case: P, E ~ N(0, 0.02^2); a running first moment M ~ N(0, 1e-3^2) and
+    second moment V = (N(0, 1e-3^2))^2 (non-negative), as after a few steps."""
+    r = _rng(seed, wid, idx, 0, KIND_ADAM)
+    p = r.standard_normal(numel, dtype=np.float32) * np.float32(0.02)
+    m = r.standard_normal(numel, dtype=np.float32) * np.float32(1e-3)
+    v = (r.standard_normal(numel, dtype=np.float32) * np.float32(1e-3)) ** 2
+    e = r.standard_normal(numel, dtype=np.float32) * np.float32(0.02)
+    return p, m, v, e
+
+
+def adamw_grad(numel: int, idx: int, step: int, seed: int = 1337, wid: int = 200):
+    """fp32 gradient of non-matrix tensor idx at a step, N(0, 1e-3^2)."""
+    return (_rng(seed, wid, idx, step, KIND_ADAM + 1)
+            .standard_normal(numel, dtype=np.float32) * np.float32(1e-3))
 
 
 def update_scales(w: Workload) -> List[float]:
