@@ -230,10 +230,25 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     assert rep.plan.last_error() == 0
 
-    # ---- timed region: device time with CUDA events, per-launch events on
-    # the launching stream for the roofline.
-    rep.plan.set_timing(True)
-    rep.plan.timing_read()  # reset
+    # One CUDA graph holds a whole step (the Muon step's launches and the
+    # EMA), captured after the warm-up so that the plan's tables are on the
+    # device; the headline replays it (eager launches with --eager).
+    graph = None
+    if not args.eager:
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                rep.step()
+        stream.wait_stream(side)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        assert rep.plan.last_error() == 0
+    run_step = graph.replay if graph is not None else rep.step
+
+    # ---- timed region: device time with CUDA events on the launching stream
     clocks = ClockSampler(local_rank)
     if world > 1:
         dist.barrier()
@@ -243,15 +258,13 @@ def run_ours(args, rank, world, local_rank):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for _ in range(args.steps):
-        rep.step()
+        run_step()
     t1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
     ms = t0.elapsed_time(t1)
-    phase = rep.plan.timing_read()
-    rep.plan.set_timing(False)
     if rep.plan.last_error() != 0:
         raise RuntimeError("device-side error during the timed region")
     if world > 1:
@@ -260,6 +273,31 @@ def run_ours(args, rank, world, local_rank):
         ms = float(t.item())
     ms_per_step = ms / args.steps
     value = world * args.steps / (ms / 1e3)
+
+    # ---- per-launch times for the roofline: the same steps launched eagerly
+    # with the plan's events between its launches (the events of a replayed
+    # graph are not harvested)
+    rep.plan.set_timing(True)
+    rep.plan.timing_read()  # reset
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        rep.step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    eager_ms = ev0.elapsed_time(ev1)
+    phase = rep.plan.timing_read()
+    rep.plan.set_timing(False)
+    if rep.plan.last_error() != 0:
+        raise RuntimeError("device-side error during the eager timing loop")
+    if world > 1:
+        t = torch.tensor([eager_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        eager_ms = float(t.item())
+    eager_value = world * args.steps / (eager_ms / 1e3)
+    del graph
 
     # ---- EMA time (own events, the EMA kernel is launched on this stream)
     e0 = torch.cuda.Event(enable_timing=True)
@@ -276,7 +314,9 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- the fused AdamW + EMA pass over the model's non-matrix parameters
     # (embeddings, vectors, scalars), each launch timed alone after an L2
-    # flush (its 0.23 GB of traffic is about the size of L2)
+    # flush by a 256 MB read (its 0.23 GB of traffic is about the size of L2;
+    # a read flush also writes back the previous launch's dirty lines before
+    # the timed one starts)
     adamw = adamw_ema_measure(w, stream, max(3, min(args.steps, 20)))
 
     # ---- end to end through the public API with host buffers: pinned
@@ -353,7 +393,9 @@ def run_ours(args, rank, world, local_rank):
                    "ema_params": sum(w.ema_numels()),
                    "ns_steps": len(w.coeffs), "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (0.9 GB of state per step)",
-                   "mode": "eager launches"},
+                   "mode": "eager launches" if args.eager
+                   else "CUDA graph replay (one graph per step)",
+                   "eager_steps_per_s": round(eager_value, 3)},
         "clocks": clk,
         "e2e": {"value": round(e2e_value, 3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4},
@@ -398,12 +440,12 @@ def adamw_ema_measure(w, stream, reps):
     hyp = type("AdamW", (), dict(lr=1e-3, beta1=0.9, beta2=0.95, eps=1e-8,
                                  weight_decay=0.0))
     run = B.adamw_ema_bind(P, G, M, V, E, hyp, w.ema_decay)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    flush = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
     for t in range(1, 4):
         run(step_now=t)
     total = 0.0
     for t in range(reps):
-        flush.zero_()
+        flush.sum()
         a0 = torch.cuda.Event(enable_timing=True)
         a1 = torch.cuda.Event(enable_timing=True)
         a0.record(stream)
@@ -502,6 +544,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", type=int, default=6)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="time eager launches instead of one CUDA graph per step")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")

@@ -239,7 +239,8 @@ typedef enum {
   MUON_KIND_NS = 5,       /* all ns_steps Newton-Schulz steps, one launch:
                              gram, poly and apply tiles of every matrix and
                              step, and the weight update of the last step  */
-  MUON_KIND_COUNT = 6
+  MUON_KIND_SCALE = 6,    /* per-matrix Frobenius scale from the partials  */
+  MUON_KIND_COUNT = 7
 } muon_kind_t;
 muon_status_t muon_plan_set_timing(muon_plan_t *plan, int32_t enable);
 muon_status_t muon_plan_timing_read(muon_plan_t *plan, int32_t *launches,

@@ -24,7 +24,7 @@ MUON_ERR_CUDA = -4
 MUON_ERR_TIMEOUT = -5
 MUON_ERR_WORKSPACE = -6
 
-KIND_NAMES = ("prologue", "gram", "poly", "apply", "final", "ns")
+KIND_NAMES = ("prologue", "gram", "poly", "apply", "final", "ns", "scale")
 
 
 class muon_matrix_t(Structure):

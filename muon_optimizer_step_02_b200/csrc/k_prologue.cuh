@@ -165,26 +165,28 @@ __device__ __forceinline__ void unpack_chunk(const ChunkRaw& c, float (&gv)[8],
 //
 // The variants are separate kernels because the one-pass register budget
 // (128 per thread at two blocks per SM) leaves no room for the other path's
-// live values, and the two-pass variant keeps three blocks per SM.  Both are persistent: as many blocks as fit on the GPU at
-// once, each taking the next work item from its own counter (items listed
-// largest first) until none is left, so that no partial last wave of blocks
-// trails the pass.
+// live values, and the two-pass variant keeps three blocks per SM.  Both are
+// persistent: as many blocks as fit on the GPU at once, block b taking items
+// b, b + grid, ... of its part of the list (items listed largest first), so
+// that no partial last wave of blocks trails the pass and no counter has to
+// be reset before it.
 template <bool kOnePass>
 __global__ void __launch_bounds__(kProThreads, kOnePass ? 2 : 3)
 muon_prologue_kernel(const MatDev* __restrict__ mats,
                      const ProItem* __restrict__ items, int n_items, HyperDev h,
-                     float* __restrict__ partials, int32_t* __restrict__ item_ctr) {
+                     float* __restrict__ partials, int32_t* __restrict__ zero, int n_zero) {
   extern __shared__ __align__(16) unsigned char pro_smem[];
   __shared__ float warp_sums[kProThreads / 32];
   __shared__ float row_sums[2][kProThreads / 32];
-  __shared__ int cur_item;
 
-  for (;;) {
+  // The step's Newton-Schulz completion counters start at zero: the previous
+  // step's Newton-Schulz kernel finished before this launch, and this step's
+  // starts after it.
+  for (int i = blockIdx.x * kProThreads + threadIdx.x; i < n_zero; i += gridDim.x * kProThreads)
+    zero[i] = 0;
+
+  for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
     __syncthreads();   // the previous item's staging and sums are consumed
-    if (threadIdx.x == 0) cur_item = atomicAdd(item_ctr, 1);
-    __syncthreads();
-    const int idx = cur_item;
-    if (idx >= n_items) break;
     const ProItem it = items[idx];
     const MatDev& md = mats[it.mat];
     const int cols = md.cols;

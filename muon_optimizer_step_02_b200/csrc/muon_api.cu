@@ -35,7 +35,7 @@ namespace {
 
 constexpr int kMaxNsSteps = 16;
 constexpr int kMaxMats = 4096;
-constexpr int kMaxLaunchesPerStep = 2;
+constexpr int kMaxLaunchesPerStep = 3;   // timed segments of one step
 constexpr int kTimingSlots = 64;
 constexpr size_t kProSmemCap = 48 * 1024;   // staging of the transposed write
 
@@ -141,11 +141,9 @@ muon_status_t layout_matrix(int rows, int cols, Geom& g, size_t& off) {
   return MUON_OK;
 }
 
-size_t counter_bytes_for(int n_mats, int steps) {
-  // the two prologue item counters (one-pass, two-pass), one count per
-  // (matrix, step, phase)
-  return (2 + static_cast<size_t>(n_mats) * 3 * std::max(steps, 1)) * sizeof(int32_t);
-}
+// Counters of one step: one completion count per (matrix, step, phase),
+// zeroed by the prologue.
+int counters_for(int n_mats, int steps) { return n_mats * 3 * std::max(steps, 1); }
 
 // Prologue work items, each with its partial-sum slot (the matrix's items
 // keep consecutive slots): the one-pass items first, then the two-pass ones,
@@ -214,7 +212,6 @@ struct muon_plan {
   size_t scale_off = 0;
   size_t counter_off = 0;
   size_t lr_slot_off = 0;
-  size_t counter_bytes = 0;
   size_t pro_smem = 0;
   int n_one = 0;       // one-pass prologue items (listed first)
   size_t pro_smem_one = 0;    // dynamic shared memory of the one-pass prologue
@@ -309,8 +306,8 @@ struct LaunchTables {
 struct StepScratch {
   float* partials;    // one per prologue item
   float* mat_scale;   // one per matrix
-  int32_t* counters;  // [item counters: 2][done: n_mats * K * 3], zeroed per step
-  size_t counter_bytes;
+  int32_t* counters;  // done: n_mats * K * 3, zeroed by the prologue
+  int n_counters;
   int n_mats;
   float* lr_slot;     // the scheduled learning rate of the step (or null)
 };
@@ -447,7 +444,8 @@ void fill_sched_matrix(SchedMatrix& s, const Geom& g) {
   s.tn = g.tn;
 }
 
-// counter reset -> prologue -> Newton-Schulz (or finisher for 0 steps).
+// prologue (which also zeroes the step's counters) -> Frobenius scale ->
+// Newton-Schulz (or the finisher for 0 steps).
 void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
                   const muon_schedule_t* sched, int32_t* step_dev,
                   const float* ns_coeffs, int32_t ns_steps, const StepScratch& sc,
@@ -474,20 +472,21 @@ void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
     hd.lr_t1 = sched->lr.t1;
     lr_dev = sc.lr_slot;
   }
-  int32_t* item_ctr = sc.counters;
-  int32_t* done = sc.counters + 2;
-  cudaMemsetAsync(sc.counters, 0, sc.counter_bytes, st);
+  int32_t* done = sc.counters;
   if (t.n_one > 0)
     muon_prologue_kernel<true><<<static_cast<unsigned>(t.pro_grid[0]), kProThreads,
                                  t.pro_smem_one, st>>>(t.mats, t.items, t.n_one, hd,
-                                                       sc.partials, item_ctr);
+                                                       sc.partials, sc.counters,
+                                                       sc.n_counters);
   if (t.n_items > t.n_one)
     muon_prologue_kernel<false><<<static_cast<unsigned>(t.pro_grid[1]), kProThreads,
                                   t.pro_smem, st>>>(
-        t.mats, t.items + t.n_one, t.n_items - t.n_one, hd, sc.partials, item_ctr + 1);
+        t.mats, t.items + t.n_one, t.n_items - t.n_one, hd, sc.partials, sc.counters,
+        sc.n_counters);
+  if (rec) rec->after(MUON_KIND_PROLOGUE);
   muon_frob_scale_kernel<<<static_cast<unsigned>((sc.n_mats + 7) / 8), 256, 0, st>>>(
       t.mats, sc.n_mats, sc.partials, hd, sc.mat_scale);
-  if (rec) rec->after(MUON_KIND_PROLOGUE);
+  if (rec) rec->after(MUON_KIND_SCALE);
 
   if (ns_steps == 0) {
     muon_final_noiter_kernel<<<static_cast<unsigned>(t.n_items), kProThreads, 0,
@@ -541,9 +540,9 @@ const char* muon_status_string(muon_status_t s) {
 }
 
 int32_t muon_step_launches(int32_t ns_steps) {
-  // one prologue kernel, the Frobenius scale kernel, then one Newton-Schulz
-  // launch for all steps (or the 0-step finisher); the counter reset is a
-  // memset, not a kernel
+  // one prologue kernel (which also zeroes the step's counters), the
+  // Frobenius scale kernel, then one Newton-Schulz launch for all steps (or
+  // the 0-step finisher); no memset
   return ns_steps < 0 ? 0 : 3;
 }
 
@@ -614,8 +613,8 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
   plan->scale_off = off;
   off = align_up(off + static_cast<size_t>(n_mats) * sizeof(float), 1024);
   plan->counter_off = off;
-  plan->counter_bytes = counter_bytes_for(n_mats, max_ns_steps);
-  off = align_up(off + plan->counter_bytes, 1024);
+  off = align_up(off + static_cast<size_t>(counters_for(n_mats, max_ns_steps)) *
+                           sizeof(int32_t), 1024);
   plan->lr_slot_off = off;   // the scheduled learning rate of a step
   off = align_up(off + sizeof(float), 1024);
   plan->ws_bytes = off;
@@ -829,7 +828,7 @@ muon_status_t step_impl(muon_plan_t* plan, const muon_matrix_t* mats,
   StepScratch sc{reinterpret_cast<float*>(ws + plan->part_off),
                  reinterpret_cast<float*>(ws + plan->scale_off),
                  reinterpret_cast<int32_t*>(ws + plan->counter_off),
-                 counter_bytes_for(plan->n_mats, ns_steps), plan->n_mats,
+                 counters_for(plan->n_mats, ns_steps), plan->n_mats,
                  reinterpret_cast<float*>(ws + plan->lr_slot_off)};
   Recorder rec(plan, st);
   enqueue_step(t, *hyper, sched, step_dev, ns_coeffs, ns_steps, sc, plan->fault, changed,
@@ -1056,8 +1055,8 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
   const size_t scale_off = off;
   off = align_up(off + static_cast<size_t>(n_mats) * sizeof(float), 1024);
   const size_t counter_off = off;
-  const size_t counter_bytes = counter_bytes_for(n_mats, ns_steps);
-  off = align_up(off + counter_bytes, 1024);
+  const int n_counters = counters_for(n_mats, ns_steps);
+  off = align_up(off + static_cast<size_t>(n_counters) * sizeof(int32_t), 1024);
   const size_t ws_bytes = off;
 
   // Device address of the array on the current device (once per device).
@@ -1135,7 +1134,7 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
                  {pro_grid_one, pro_grid_two}, clusters};
   StepScratch sc{reinterpret_cast<float*>(ws + part_off),
                  reinterpret_cast<float*>(ws + scale_off),
-                 reinterpret_cast<int32_t*>(ws + counter_off), counter_bytes, n_mats,
+                 reinterpret_cast<int32_t*>(ws + counter_off), n_counters, n_mats,
                  nullptr};
   enqueue_step(t, *hyper, nullptr, nullptr, ns_coeffs, ns_steps, sc, 0, true, st, nullptr);
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
