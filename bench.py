@@ -40,18 +40,24 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
                   "bf16_tflops_sustained": 1400.0}
 
 
-def kernel_source_hash() -> str:
-    """sha256 over the CUDA sources, to tell whether a recorded ncu traffic
-    figure still belongs to the kernels being timed."""
-    import glob
+# CUDA sources each recorded kernel is built from (its own code, the shared
+# PTX wrappers and tables, and the host-built schedule that orders its work)
+KERNEL_SOURCES = {
+    "ns_mega_pair_kernel": ("k_ns_mega.cuh", "k_ns_common.cuh", "sm100_ptx.cuh",
+                            "muon_types.cuh", "schedule.h"),
+}
+
+
+def kernel_source_hash(kernel: str = "ns_mega_pair_kernel") -> str:
+    """sha256 over the CUDA sources of `kernel`, to tell whether a recorded
+    ncu traffic figure still belongs to the kernel being timed."""
     import hashlib
     h = hashlib.sha256()
-    pat = os.path.join(ROOT, "muon_optimizer_step_02_b200", "csrc", "*")
-    for f in sorted(glob.glob(pat)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(os.path.basename(f).encode())
-            with open(f, "rb") as fh:
-                h.update(fh.read())
+    for name in KERNEL_SOURCES[kernel]:
+        path = os.path.join(ROOT, "muon_optimizer_step_02_b200", "csrc", name)
+        h.update(name.encode())
+        with open(path, "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()
 
 
@@ -68,7 +74,7 @@ def recorded_traffic(kernel: str, workload: int):
     rec = doc.get(kernel)
     if not rec or rec.get("workload") != workload:
         return None
-    if rec.get("source_sha256") != kernel_source_hash():
+    if kernel not in KERNEL_SOURCES or rec.get("source_sha256") != kernel_source_hash(kernel):
         return None
     return rec.get("dram_bytes_per_launch")
 

@@ -28,7 +28,7 @@
 
 namespace muonb200 {
 
-constexpr int kAdamMaxSegs = 160;   // 160 x 56 bytes of kernel parameters
+constexpr int kAdamMaxSegs = 480;   // 480 x 56 bytes: 27 KB of kernel parameters (limit 32 KB)
 constexpr int kAdamThreads = 256;
 
 struct AdamSeg {

@@ -126,11 +126,27 @@ def test_device_step_counter_and_graph_replay():
     del graph
 
 
+def test_many_tensors_take_several_launches():
+    """More tensors than one launch's segment table (480): the call splits
+    them over launches; every tensor still matches the oracle."""
+    import torch
+    from muon_optimizer_step_02_b200 import binding as B
+    sizes = [(7 * i) % 37 for i in range(500)]
+    st = State(sizes, seed=99)
+    run = B.adamw_ema_bind(st.P, st.G, st.M, st.V, st.E, H, DECAY)
+    st.set_grads(1)
+    before = st.snapshot()
+    run(step_now=1)
+    torch.cuda.synchronize()
+    _check(st, before, 1, 1)
+
+
 def test_adamw_launch_count():
     from muon_optimizer_step_02_b200 import binding as B
     assert B.adamw_ema_launches(len(SIZES)) == 1
     assert B.adamw_ema_launches(len(SIZES), True) == 2
-    assert B.adamw_ema_launches(161) == 2
+    assert B.adamw_ema_launches(481) == 2
+    assert B.adamw_ema_launches(212) == 1     # the 11L model's non-matrix tensors
 
 
 def test_adamw_argument_errors():
