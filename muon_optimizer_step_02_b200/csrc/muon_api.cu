@@ -789,6 +789,9 @@ muon_status_t step_impl(muon_plan_t* plan, const muon_matrix_t* mats,
   const bool resched = ns_steps > 0 && ns_steps != plan->sched_steps;
   if (changed || resched) {
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    // The host copy of the table already holds this call's pointers: until a
+    // call uploads it, the device copy is stale.
+    if (changed) plan->h_valid = false;
     if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return MUON_ERR_CUDA;
     // A host-to-device table copy cannot be captured from pageable memory:
     // run one call with the same buffers and step count before capturing.
