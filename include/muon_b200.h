@@ -220,6 +220,16 @@ muon_status_t adamw_ema_batched(const adamw_tensor_t *tensors, int32_t n_tensors
  * last call, MUON_ERR_CUDA on a CUDA error, MUON_OK otherwise. */
 muon_status_t muon_get_last_error(muon_plan_t *plan, muon_stream_t stream);
 
+/* Enqueues on `stream` a copy of the plan's device error word into
+ * *host_word (host memory; pinned for the copy to be asynchronous) without
+ * synchronising, for loops that check each step's status a step later.
+ * Non-zero means a kernel gave up on a bounded wait (MUON_ERR_TIMEOUT); the
+ * word stays set until muon_get_last_error reads and clears it.  Returns
+ * MUON_ERR_INVALID_ARG for a NULL argument, MUON_ERR_CUDA if the copy cannot
+ * be enqueued. */
+muon_status_t muon_plan_error_async(const muon_plan_t *plan, int32_t *host_word,
+                                    muon_stream_t stream);
+
 /* Static description of a status code. */
 const char *muon_status_string(muon_status_t status);
 

@@ -122,6 +122,8 @@ def lib():
     L.adamw_ema_batched.restype = c_int32
     L.adamw_ema_launches.argtypes = [c_int32, c_int32]
     L.adamw_ema_launches.restype = c_int32
+    L.muon_plan_error_async.argtypes = [c_void_p, c_void_p, c_void_p]
+    L.muon_plan_error_async.restype = c_int32
     L.muon_step_launches.argtypes = [c_int32]
     L.muon_step_launches.restype = c_int32
     L.muon_plan_step_launches.argtypes = [c_void_p, c_int32]
@@ -274,6 +276,18 @@ class MuonPlan:
 
     def last_error(self, stream=None) -> int:
         return int(lib().muon_get_last_error(self._h, _stream_handle(stream)))
+
+    def error_async(self, host_word, stream=None):
+        """Enqueues a copy of the device error word into `host_word` (a
+        one-element int32 CPU tensor, pinned for the copy to be asynchronous);
+        read it after the stream has passed this point."""
+        import torch
+        if host_word.dtype != torch.int32 or host_word.device.type != "cpu" or \
+                host_word.numel() < 1:
+            raise ValueError("host_word must be an int32 CPU tensor")
+        _check(lib().muon_plan_error_async(self._h, host_word.data_ptr(),
+                                           _stream_handle(stream)),
+               "muon_plan_error_async")
 
     def step_launches(self, ns_steps: int) -> int:
         return int(lib().muon_plan_step_launches(self._h, int(ns_steps)))

@@ -845,6 +845,17 @@ muon_status_t step_impl(muon_plan_t* plan, const muon_matrix_t* mats,
 
 extern "C" {
 
+muon_status_t muon_plan_error_async(const muon_plan_t* plan, int32_t* host_word,
+                                    muon_stream_t stream) {
+  if (!plan || !host_word) return MUON_ERR_INVALID_ARG;
+  if (cudaMemcpyAsync(host_word, plan->d_err, sizeof(int32_t), cudaMemcpyDeviceToHost,
+                      static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return MUON_ERR_CUDA;
+  }
+  return MUON_OK;
+}
+
 muon_status_t muon_step_batched(muon_plan_t* plan, const muon_matrix_t* mats,
                                 const muon_hyper_t* hyper,
                                 const float* ns_coeffs, int32_t ns_steps,

@@ -24,6 +24,10 @@ def test_bounded_wait_timeout_is_reported_and_recoverable():
     g.plan.set_fault(1)
     t0 = time.time()
     g.step(g.grads(0))
+    word = torch.zeros(1, dtype=torch.int32).pin_memory()
+    g.plan.error_async(word)              # no synchronisation
+    torch.cuda.current_stream().synchronize()
+    assert int(word[0]) != 0              # the asynchronous copy saw the error word
     status = g.plan.last_error()          # synchronises the stream
     elapsed = time.time() - t0
     assert status == B.MUON_ERR_TIMEOUT
@@ -35,3 +39,7 @@ def test_bounded_wait_timeout_is_reported_and_recoverable():
     torch.cuda.synchronize()
     g2 = GpuMuon(w)
     check_step(g2, 0, [0, 1])
+    word[0] = 7
+    g2.plan.error_async(word)
+    torch.cuda.current_stream().synchronize()
+    assert int(word[0]) == 0
