@@ -33,7 +33,7 @@ per-matrix algorithm below is the method's stated definition, taken in order:
   8. update          W' = W (1 - lr*wd) - lr*scale*O
   9. EMA             E' = d*E + (1-d)*P
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 the "sum" Nesterov form; epsilons added to the norm, not inside the square
 root; the row norm taken over rows of the stored (out x in) weight before any
 transpose; transpose iff rows > cols; weight decay applied to the
