@@ -105,3 +105,86 @@ def test_sharded_step_matches_single_process():
         assert t == 2.0            # max over ranks of 1.0 + rank
         for a, b in zip(Ws, W):
             np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
+
+
+def test_flat_layout_is_owner_ordered_and_aligned():
+    shapes = wl.workload(2).shapes
+    for world in (1, 2, 8):
+        L = sharding.ShardLayout(shapes, world)
+        assert L.owner == sharding.partition_matrices(shapes, world)
+        spans = []
+        for i, (r, c) in enumerate(shapes):
+            o = L.owner[i]
+            assert o * L.seg <= L.offset[i] and L.offset[i] + r * c <= (o + 1) * L.seg
+            assert L.offset[i] % 8 == 0
+            spans.append((L.offset[i], L.offset[i] + r * c))
+        spans.sort()
+        assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))   # no overlap
+        assert L.numel() == world * L.seg
+
+
+def _flat_worker(rank, world, port, q):
+    import oracle.muon_oracle as mo
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            init_method=f"tcp://127.0.0.1:{port}")
+    try:
+        shapes = [(48, 32), (32, 48), (40, 40), (16, 64), (64, 16), (24, 24), (8, 100)]
+        h = wl.Hyper(momentum=0.9, lr=0.05, weight_decay=0.1)
+        coeffs = [wl.FIXED_QUINTIC] * 3
+        w = wl.custom(shapes, h, coeffs, grad_std=1.0, wid=401)
+        L = sharding.ShardLayout(shapes, world, 3)
+        W_flat = torch.zeros(L.numel(), dtype=torch.float64)
+        for i, v in enumerate(L.views(W_flat)):
+            v.copy_(torch.from_numpy(wl.weight(w, i).astype(np.float64)))
+        M_seg = torch.zeros(L.seg, dtype=torch.float64)
+        G_seg = torch.zeros(L.seg, dtype=torch.float64)
+        hyp = mo.MuonHyper(momentum=h.momentum, lr=h.lr, weight_decay=h.weight_decay)
+
+        def step_fn(Wv, Mv, Gv):
+            for a, m, g in zip(Wv, Mv, Gv):
+                Wn, Mn, _ = mo.muon_step(a.numpy(), m.numpy(), g.numpy(), hyp, coeffs, 1.0)
+                a.copy_(torch.from_numpy(Wn))
+                m.copy_(torch.from_numpy(Mn))
+
+        for step in range(2):
+            G_flat = torch.zeros(L.numel(), dtype=torch.float64)
+            share = 0.25 if rank == 0 else 0.75
+            for i, v in enumerate(L.views(G_flat)):
+                g = wl.bf16_bits_to_f32(wl.grad_bits(w, i, step)).astype(np.float64)
+                v.copy_(torch.from_numpy(g * share))
+            sharding.sharded_step_flat(L, W_flat, M_seg, G_flat, G_seg, rank, step_fn)
+        q.put((rank, [v.numpy().copy() for v in L.views(W_flat)]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_flat_sharded_step_matches_single_process():
+    import oracle.muon_oracle as mo
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_flat_worker, args=(r, world, port, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    shapes = [(48, 32), (32, 48), (40, 40), (16, 64), (64, 16), (24, 24), (8, 100)]
+    h = wl.Hyper(momentum=0.9, lr=0.05, weight_decay=0.1)
+    coeffs = [wl.FIXED_QUINTIC] * 3
+    w = wl.custom(shapes, h, coeffs, grad_std=1.0, wid=401)
+    hyp = mo.MuonHyper(momentum=h.momentum, lr=h.lr, weight_decay=h.weight_decay)
+    W = [wl.weight(w, i).astype(np.float64) for i in range(len(shapes))]
+    M = [np.zeros_like(x) for x in W]
+    for step in range(2):
+        for i in range(len(shapes)):
+            G = wl.bf16_bits_to_f32(wl.grad_bits(w, i, step)).astype(np.float64)
+            W[i], M[i], _ = mo.muon_step(W[i], M[i], G, hyp, coeffs, 1.0)
+    for rank, Ws in out:
+        for a, b in zip(Ws, W):
+            np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
