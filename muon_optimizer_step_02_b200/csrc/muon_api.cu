@@ -65,10 +65,10 @@ EncodeTiledFn get_encode_fn() {
 }
 
 // bf16 matrix of `rows` x `cols` elements with leading dimension `ld`,
-// boxes of box_cols x box_rows (128-byte swizzle for operand loads, none for
-// the epilogue's 32 x 32 stores).
+// boxes of box_cols x box_rows, 128-byte swizzle (the tensor-core operand
+// layout in shared memory).
 bool encode_bf16_2d(CUtensorMap* tm, void* base, int rows, int cols, int ld,
-                    int box_cols, int box_rows, bool swizzle = true) {
+                    int box_cols, int box_rows) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols),
@@ -79,7 +79,7 @@ bool encode_bf16_2d(CUtensorMap* tm, void* base, int rows, int cols, int ld,
   cuuint32_t estr[2] = {1, 1};
   return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -345,16 +345,13 @@ bool fill_workspace_fields(MatDev& d, const Geom& g, char* ws) {
   for (int b = 0; b < 2; ++b) {
     d.x[b] = reinterpret_cast<__nv_bfloat16*>(ws + g.x_off[b]);
     if (!encode_bf16_2d(&d.tm_xk[b], d.x[b], g.m, g.n, g.ldx, kTileK, kTileM) ||
-        !encode_bf16_2d(&d.tm_xn[b], d.x[b], g.m, g.n, g.ldx, 64, kTileK) ||
-        !encode_bf16_2d(&d.tm_xs[b], d.x[b], g.m, g.n, g.ldx, 32, 32, false))
+        !encode_bf16_2d(&d.tm_xn[b], d.x[b], g.m, g.n, g.ldx, 64, kTileK))
       return false;
   }
   d.a = reinterpret_cast<__nv_bfloat16*>(ws + g.a_off);
   d.b = reinterpret_cast<__nv_bfloat16*>(ws + g.b_off);
   if (!encode_bf16_2d(&d.tm_a, d.a, g.m, g.m, g.lda, kTileK, kTileM) ||
-      !encode_bf16_2d(&d.tm_b, d.b, g.m, g.m, g.lda, kTileK, kTileM) ||
-      !encode_bf16_2d(&d.tm_as, d.a, g.m, g.m, g.lda, 32, 32, false) ||
-      !encode_bf16_2d(&d.tm_bs, d.b, g.m, g.m, g.lda, 32, 32, false))
+      !encode_bf16_2d(&d.tm_b, d.b, g.m, g.m, g.lda, kTileK, kTileM))
     return false;
   d.rows = g.rows;
   d.cols = g.cols;
