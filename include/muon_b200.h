@@ -268,9 +268,13 @@ int32_t ema_update_launches(int32_t n_tensors);
  * advanced). */
 int32_t adamw_ema_launches(int32_t n_tensors, int32_t with_step_dev);
 
-/* Test hook: fault 1 makes the tensor-core kernel's load warp skip one
+/* Test hooks.  Fault 1 makes the tensor-core kernel's load warp skip one
  * stage of its first tile in block 0, so that the consumer's bounded wait
- * runs out and the timeout path is exercised.  0 turns it off. */
+ * runs out and the timeout path is exercised (MUON_ERR_TIMEOUT from
+ * muon_get_last_error).  Fault 2 asks for more dynamic shared memory than the
+ * tensor-core kernel was set up for, so that the runtime refuses its launch
+ * and the step call returns MUON_ERR_CUDA (no kernel of it runs; the earlier
+ * launches of the call do).  0 turns them off. */
 muon_status_t muon_plan_set_fault(muon_plan_t *plan, int32_t fault);
 
 /* ABI version (major * 100 + minor). */

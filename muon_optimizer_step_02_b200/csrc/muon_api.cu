@@ -10,6 +10,7 @@
 // No device memory is allocated after muon_plan_create.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -470,6 +471,7 @@ void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
     lr_dev = sc.lr_slot;
   }
   int32_t* done = sc.counters;
+  nvtxRangePushA("muon.prologue");
   if (t.n_one > 0)
     muon_prologue_kernel<true><<<static_cast<unsigned>(t.pro_grid[0]), kProThreads,
                                  t.pro_smem_one, st>>>(t.mats, t.items, t.n_one, hd,
@@ -480,9 +482,12 @@ void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
                                   t.pro_smem, st>>>(
         t.mats, t.items + t.n_one, t.n_items - t.n_one, hd, sc.partials, sc.counters,
         sc.n_counters);
+  nvtxRangePop();
   if (rec) rec->after(MUON_KIND_PROLOGUE);
+  nvtxRangePushA("muon.frobenius_scale");
   muon_frob_scale_kernel<<<static_cast<unsigned>((sc.n_mats + 7) / 8), 256, 0, st>>>(
       t.mats, sc.n_mats, sc.partials, hd, sc.mat_scale);
+  nvtxRangePop();
   if (rec) rec->after(MUON_KIND_SCALE);
 
   if (ns_steps == 0) {
@@ -513,7 +518,12 @@ void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
   p.eps_frob = h.eps_frob;
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = pair_launch_config(t.clusters, st, attr);
+  // test hook 2: more dynamic shared memory than the kernel was set up for,
+  // so that the runtime refuses the launch (no kernel runs)
+  if (fault == 2) cfg.dynamicSmemBytes = kMegaSmemBytes + 64 * 1024;
+  nvtxRangePushA("muon.newton_schulz");
   cudaLaunchKernelEx(&cfg, ns_mega_pair_kernel, p);
+  nvtxRangePop();
   if (rec) rec->after(MUON_KIND_NS);
 }
 
@@ -685,7 +695,7 @@ void muon_plan_destroy(muon_plan_t* plan) {
 }
 
 muon_status_t muon_plan_set_fault(muon_plan_t* plan, int32_t fault) {
-  if (!plan || fault < 0 || fault > 1) return MUON_ERR_INVALID_ARG;
+  if (!plan || fault < 0 || fault > 2) return MUON_ERR_INVALID_ARG;
   plan->fault = fault;
   return MUON_OK;
 }
@@ -914,7 +924,9 @@ muon_status_t ema_update_batched(float* const* ema, const float* const* params,
     if (units == 0) continue;
     const long long want = (units + kEmaThreads - 1) / kEmaThreads;
     const unsigned grid = static_cast<unsigned>(std::min<long long>(want, 8ll * sms));
+    nvtxRangePushA("muon.ema");
     ema_update_kernel<<<grid, kEmaThreads, 0, st>>>(p);
+    nvtxRangePop();
   }
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
@@ -971,7 +983,9 @@ muon_status_t adamw_ema_batched(const adamw_tensor_t* tensors, int32_t n_tensors
     // (launched even when empty, so that the launch count is fixed)
     const long long want = std::max(1ll, (units + kAdamThreads - 1) / kAdamThreads);
     const unsigned grid = static_cast<unsigned>(std::min<long long>(want, 8ll * sms));
+    nvtxRangePushA("muon.adamw_ema");
     adamw_ema_kernel<<<grid, kAdamThreads, 0, st>>>(a);
+    nvtxRangePop();
   }
   if (step_dev) adamw_step_advance_kernel<<<1, 1, 0, st>>>(step_dev);
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;

@@ -43,3 +43,24 @@ def test_bounded_wait_timeout_is_reported_and_recoverable():
     g2.plan.error_async(word)
     torch.cuda.current_stream().synchronize()
     assert int(word[0]) == 0
+
+
+def test_refused_launch_is_reported_and_recoverable():
+    """Test hook 2: the runtime refuses the tensor-core kernel's launch (more
+    shared memory than it was set up for).  The step call returns
+    MUON_ERR_CUDA at once, no device error is left behind, and the next step
+    on a fresh state matches the oracle."""
+    import torch
+    from muon_optimizer_step_02_b200 import binding as B
+    h = wl.Hyper(momentum=0.95, lr=0.02, weight_decay=0.1)
+    w = wl.custom([(256, 512), (512, 256)], h, [wl.FIXED_QUINTIC] * 5, wid=501)
+    g = GpuMuon(w)
+    g.plan.set_fault(2)
+    with pytest.raises(B.MuonError) as err:
+        g.step(g.grads(0))
+    assert err.value.status == B.MUON_ERR_CUDA
+    g.plan.set_fault(0)
+    torch.cuda.synchronize()
+    assert g.plan.last_error() == B.MUON_OK
+    g2 = GpuMuon(w)
+    check_step(g2, 0, [0, 1])
