@@ -22,6 +22,13 @@
  *    the readings this library implements.
  *  - ema_update_batched: E' = d E + (1 - d) P for every parameter tensor
  *    (PR #1893, same table, row "EMA": EMA_DECAY=0.9965).
+ *  - muon_step_batched_sched: the Muon step with momentum and learning rate
+ *    taken from linear ramps at a step number held in device memory (PR
+ *    #1893, same table, row "Optimizer": momentum warm-up from 0.92 over 1500
+ *    steps).
+ *  - adamw_ema_batched: AdamW of the non-matrix tensors and the EMA of their
+ *    new values in one pass (PR #1893, same table, row "Optimizer": AdamW on
+ *    embeddings/scalars).
  *
  * Conventions for every call:
  *  - Pointers named device point to device memory; pointers to structs and
@@ -32,7 +39,8 @@
  *    muon_plan_destroy).
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *    stream) and the calls return without synchronising, except
- *    muon_get_last_error, which synchronises `stream`.
+ *    muon_get_last_error (synchronises `stream`), muon_plan_timing_read and
+ *    muon_plan_destroy (synchronise the device).
  *  - Argument, shape and alignment errors are detected on the host and
  *    returned before anything is enqueued.  Launch failures return
  *    MUON_ERR_CUDA.  A device-side wait that exceeds its time limit (about one
