@@ -133,3 +133,19 @@ def test_schedule_argument_errors():
     assert call(ctypes.byref(ok), step_dev.data_ptr() + 2) == B.MUON_ERR_ALIGNMENT
     torch.cuda.synchronize()
     assert int(step_dev[0].item()) == 0          # nothing was enqueued
+
+
+def test_scheduled_step_without_newton_schulz():
+    """K = 0: the finishing kernel takes the scheduled learning rate too."""
+    import torch
+    w = wl.custom([(96, 160), (160, 96)], H, [], wid=124)
+    g = GpuMuon(w)
+    step_dev = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for t in range(3):
+        W0 = [x.cpu().numpy().astype(np.float64) for x in g.W]
+        M0 = [x.cpu().numpy().astype(np.float64) for x in g.M]
+        _sched_step(g, g.grads(t), step_dev, (MU, LR))
+        torch.cuda.synchronize()
+        assert g.plan.last_error() == 0
+        _check_against_oracle(g, t, W0, M0, t, (MU, LR))
+    assert int(step_dev.item()) == 3
