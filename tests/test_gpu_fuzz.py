@@ -1,0 +1,40 @@
+"""Seeded random cases against the fp64 oracle: random shapes (1..700 rows
+and columns, both orientations, aligned and not), random switches and step
+counts, several matrices per plan, two consecutive steps."""
+import numpy as np
+import pytest
+
+from gpu_harness import GpuMuon, check_step
+from muon_optimizer_step_02_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+Q5 = [wl.FIXED_QUINTIC] * 5
+
+
+def _case(seed):
+    rng = np.random.default_rng(seed)
+    n = int(rng.integers(1, 5))
+    shapes = []
+    for _ in range(n):
+        r = int(rng.integers(1, 701))
+        c = int(rng.integers(1, 701))
+        if rng.random() < 0.5:            # often a multiple of 8 (one-pass rows)
+            c = max(8, c // 8 * 8)
+        shapes.append((r, c))
+    k = int(rng.integers(0, 6))
+    h = wl.Hyper(momentum=float(rng.uniform(0.5, 0.99)),
+                 lr=float(rng.uniform(0.005, 0.05)),
+                 weight_decay=float(rng.uniform(0.0, 0.2)),
+                 nesterov=bool(rng.random() < 0.8), eq_r=bool(rng.random() < 0.8))
+    return shapes, h, Q5[:k]
+
+
+@pytest.mark.parametrize("seed", list(range(40)))
+def test_random_case_matches_oracle(seed):
+    shapes, h, coeffs = _case(1000 + seed)
+    w = wl.custom(shapes, h, coeffs, grad_std=float(10.0 ** (seed % 3 - 2)),
+                  wid=600 + seed)
+    g = GpuMuon(w)
+    for step in range(2):
+        check_step(g, step, list(range(w.n_mats)))
