@@ -28,6 +28,10 @@ __device__ __forceinline__ float warp_allreduce_sum(float v) {
   return v;
 }
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }
@@ -174,7 +178,8 @@ template <bool kOnePass>
 __global__ void __launch_bounds__(kProThreads, kOnePass ? 2 : 3)
 muon_prologue_kernel(const MatDev* __restrict__ mats,
                      const ProItem* __restrict__ items, int n_items, HyperDev h,
-                     float* __restrict__ partials, int32_t* __restrict__ zero, int n_zero) {
+                     float* __restrict__ partials, int32_t* __restrict__ zero, int n_zero,
+                     int prefetch) {
   extern __shared__ __align__(16) unsigned char pro_smem[];
   __shared__ float warp_sums[kProThreads / 32];
   __shared__ float row_sums[2][kProThreads / 32];
@@ -218,6 +223,20 @@ muon_prologue_kernel(const MatDev* __restrict__ mats,
         for (int j = 0; j < 4; ++j) {
           const int p0 = (wi * 4 + j) * 256 + lane * 8;
           if (act && p0 < cols) load_chunk_vec(g, mo, p0, raw[j]);
+        }
+        // The next pass's row of this warp goes into L2 while this one is
+        // processed (when the host asks for it): one prefetch per 128-byte
+        // line of G (every 8th lane) and of M (every 4th lane).
+        if (prefetch && r + rpp < it.nrows) {
+          const size_t nbase = static_cast<size_t>(it.row0 + r + rpp) * cols;
+  #pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int p0 = (wi * 4 + j) * 256 + lane * 8;
+            if (p0 < cols) {
+              if ((lane & 7) == 0) prefetch_l2(md.g + nbase + p0);
+              if ((lane & 3) == 0) prefetch_l2(md.mom + nbase + p0);
+            }
+          }
         }
         float u[4][8];
         float ss = 0.f;
