@@ -7,7 +7,7 @@ One step = muon_step_batched over the 66 matrices of the 11L x 512d GPT
 (K = 5 fixed-quintic Newton-Schulz steps, momentum 0.99, lr 0.022, wd 0.105,
 MuonEq-R) followed by ema_update_batched over every parameter of the same
 model (38,071,388 fp32, decay 0.9965): every row of the hot path.  Inputs are
-synthetic (seeded), resident in HBM and larger than L2 (0.9 GB of state).
+synthetic (seeded), resident in HBM and larger than L2 (about 0.67 GB for the 11L set).
 
 For N > 1 it runs under torch.distributed.run, one rank per GPU; each rank
 steps its own replica (weak scaling, no collective on the data path); the
@@ -216,6 +216,12 @@ class Workload:
         return {"gram": gram, "poly": poly, "apply": gram,
                 "ns": k * (2 * gram + poly)}
 
+    def resident_bytes(self) -> int:
+        """Device bytes the step reads or writes: W, M, G, the plan's
+        workspace, the averages and the non-matrix parameters."""
+        ts = self.W + self.M + self.G + self.E + self.extra + [self.ws]
+        return sum(t.numel() * t.element_size() for t in ts)
+
     def state_bytes(self):
         elems = self.w.numel()
         return {"prologue": 12 * elems,  # G 2 + M 4+4 + X~ 2
@@ -398,6 +404,10 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return None
 
+    # ---- yardstick: the same Newton-Schulz work as torch/cuBLAS GEMMs
+    yard_ms = (torch_ns_yardstick(w, stream, max(3, min(args.steps, 20)))
+               if not args.no_yardstick else None)
+
     # ---- roofline of the dominant kernel
     flops = rep.ns_flops_by_kind()
     ns_kinds = ("gram", "poly", "apply", "ns")
@@ -442,7 +452,8 @@ def run_ours(args, rank, world, local_rank):
                    "matrix_params": w.numel(),
                    "ema_params": sum(w.ema_numels()),
                    "ns_steps": len(w.coeffs), "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (0.9 GB of state per step)",
+                   "l2": f"inputs larger than L2 ({rep.resident_bytes() / 1e9:.2f} GB "
+                         "resident, all of it read or written every step)",
                    "mode": "eager launches" if args.eager
                    else "CUDA graph replay (one graph per step)",
                    "eager_steps_per_s": round(eager_value, 3)},
@@ -456,7 +467,10 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roof,
         "ns": {"tflops": round(ns_tflops, 2) if ns_tflops else None,
                "frac_of_sustained": round(ns_tflops / sustained, 4)
-               if ns_tflops else None, "ms_per_step": round(ns_ms, 4)},
+               if ns_tflops else None, "ms_per_step": round(ns_ms, 4),
+               "issued_tflops": round(ns_issued_flops(w) / (ns_ms / 1e3) / 1e12, 2)
+               if ns_ms > 0 else None,
+               "issued_flops_per_launch": ns_issued_flops(w)},
         "prologue_gbs": round(rep.state_bytes()["prologue"] / (pro_ms / 1e3) / 1e9, 1)
         if pro_ms > 0 else None,
         "ema": {"gbs": round(ema_gbs, 1) if ema_gbs else None,
@@ -464,6 +478,14 @@ def run_ours(args, rank, world, local_rank):
                 "ms": round(ema_ms, 4) if ema_ms else None},
         "breakdown": breakdown,
     }
+    if yard_ms is not None:
+        line["yardstick"] = {
+            "impl": "torch.bmm + baddbmm (cuBLAS), bf16, dense products, "
+                    "grouped by shape, one CUDA graph",
+            "work": "the Newton-Schulz steps only (no prologue, scale or W update)",
+            "ns_ms": round(yard_ms, 4),
+            "tflops": round(flops["ns"] / (yard_ms / 1e3) / 1e12, 2),
+            "fused_speedup": round(yard_ms / ns_ms, 3) if ns_ms > 0 else None}
     if adamw is not None:
         a_ms, a_params = adamw
         a_gbs = 36 * a_params / (a_ms / 1e3) / 1e9
@@ -508,6 +530,77 @@ def adamw_ema_measure(w, stream, reps):
         total += a0.elapsed_time(a1)
     del flush
     return total / reps, sum(numels)
+
+
+def ns_issued_flops(w: wl.Workload) -> int:
+    """FLOPs the tensor cores issue in one Newton-Schulz launch: whole
+    256 x 256 pair tiles and 64-deep K blocks (the ragged edges zero-padded),
+    the gram and polynomial products on the upper pair tiles only."""
+    def cdiv(a, b):
+        return -(-a // b)
+    blocks = 0
+    for r, c in w.shapes:
+        m, n = min(r, c), max(r, c)
+        t2, tn = cdiv(m, 256), cdiv(n, 256)
+        sym = t2 * (t2 + 1) // 2
+        blocks += sym * cdiv(n, 64) + sym * cdiv(m, 64) + t2 * tn * cdiv(m, 64)
+    return blocks * 2 * 256 * 256 * 64 * len(w.coeffs)
+
+
+def torch_ns_yardstick(w: wl.Workload, stream, reps: int):
+    """The same Newton-Schulz work as cuBLAS batched GEMMs through torch, as a
+    yardstick for the fused kernel (not part of the library): per group of
+    equal working shapes, every step runs A = X X^T, B = b A + c A A and
+    X <- a X + B X (bmm and two baddbmm, bf16 in and out, the full dense
+    products), all steps replayed from one CUDA graph.  Returns the device
+    time of one replay in ms."""
+    import torch
+    groups = {}
+    for r, c in w.shapes:
+        key = (min(r, c), max(r, c))
+        groups[key] = groups.get(key, 0) + 1
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(7)
+    bufs = []
+    for (m, n), cnt in groups.items():
+        x0 = (torch.randn(cnt, m, n, device="cuda", generator=gen)
+              / float(np.sqrt(m * n))).to(torch.bfloat16)
+        bufs.append((x0, torch.empty_like(x0), torch.empty_like(x0),
+                     torch.empty(cnt, m, m, device="cuda", dtype=torch.bfloat16),
+                     torch.empty(cnt, m, m, device="cuda", dtype=torch.bfloat16)))
+
+    def ns():
+        cur = [b[0] for b in bufs]
+        for k, (a, b, c) in enumerate(w.coeffs):
+            for i, (_, x1, x2, A, Bm) in enumerate(bufs):
+                x = cur[i]
+                torch.bmm(x, x.transpose(1, 2), out=A)
+                torch.baddbmm(A, A, A, beta=b, alpha=c, out=Bm)
+                nxt = x1 if k % 2 == 0 else x2
+                torch.baddbmm(x, Bm, x, beta=a, alpha=1.0, out=nxt)
+                cur[i] = nxt
+
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        ns()                                   # cuBLAS handles and workspaces
+        side.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            ns()
+    stream.wait_stream(side)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    y0 = torch.cuda.Event(enable_timing=True)
+    y1 = torch.cuda.Event(enable_timing=True)
+    y0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    y1.record(stream)
+    torch.cuda.synchronize()
+    del graph
+    return y0.elapsed_time(y1) / reps
 
 
 # --------------------------------------------------------------------------
@@ -597,6 +690,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", type=int, default=6)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-yardstick", action="store_true",
+                    help="skip timing the same Newton-Schulz work as torch/cuBLAS GEMMs")
     ap.add_argument("--eager", action="store_true",
                     help="time eager launches instead of one CUDA graph per step")
     args = ap.parse_args()
