@@ -728,6 +728,16 @@ def main():
         line["cpu_baseline"] = {"value": round(1.0 / s, 6), "unit": UNIT,
                                 "cores": threads, "kind": "oracle",
                                 "sample": desc}
+        # the same oracle on one host thread (BLAS limited to one thread),
+        # over a smaller sample
+        try:
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                s1, desc1, _ = oracle_sample(wl.workload(args.workload), budget / 3)
+            line["cpu_baseline"]["one_thread"] = {"value": round(1.0 / s1, 6),
+                                                  "unit": UNIT, "sample": desc1}
+        except ImportError:
+            pass
     print(json.dumps(line), flush=True)
 
 
