@@ -244,13 +244,19 @@ class MuonPlan:
                           float(hyper.weight_decay), float(hyper.eps_row),
                           float(hyper.eps_frob), int(bool(hyper.nesterov)),
                           int(bool(hyper.eq_r)))
+        if any(len(row) != 3 for row in coeffs):
+            raise ValueError("coeffs: one (a, b, c) row per Newton-Schulz step")
         flat = [float(v) for row in coeffs for v in row]
         k = len(flat) // 3
         carr = (c_float * max(len(flat), 1))(*flat)
         _check_tensor(workspace, torch.uint8, (workspace.numel(),),
                       "workspace")
-        h, hp_ref = self._h, ctypes.byref(hp)
+        hp_ref = ctypes.byref(hp)
         ws_ptr, ws_n = workspace.data_ptr(), workspace.numel()
+        # The callable holds the plan (so that it outlives every bound call)
+        # and reads its handle at call time (so that a closed plan raises
+        # instead of handing a freed handle to the library).
+        plan = self
         keep = (mats, hp, carr, weights, momenta, grads, update_out, workspace)
         if schedule is not None:
             if step_dev is None:
@@ -263,16 +269,22 @@ class MuonPlan:
 
             def run_sched(stream=None):
                 _ = keep
-                _check(fn_s(h, mats, hp_ref, sch_ref, sp, carr, k, ws_ptr, ws_n,
-                            _stream_handle(stream)), "muon_step_batched_sched")
+                _check(fn_s(plan._live_handle(), mats, hp_ref, sch_ref, sp, carr,
+                            k, ws_ptr, ws_n, _stream_handle(stream)),
+                       "muon_step_batched_sched")
             return run_sched
         fn = lib().muon_step_batched
 
         def run(stream=None):
             _ = keep
-            _check(fn(h, mats, hp_ref, carr, k, ws_ptr, ws_n,
+            _check(fn(plan._live_handle(), mats, hp_ref, carr, k, ws_ptr, ws_n,
                       _stream_handle(stream)), "muon_step_batched")
         return run
+
+    def _live_handle(self):
+        if self._h is None:
+            raise MuonError(MUON_ERR_INVALID_ARG, "the plan has been closed")
+        return self._h
 
     def last_error(self, stream=None) -> int:
         return int(lib().muon_get_last_error(self._h, _stream_handle(stream)))

@@ -109,3 +109,14 @@ def test_ema_validation_catches_misalignment(L):
     n3 = (ctypes.c_int64 * 1)(8)
     assert L.ema_update_batched(e, p, n3, 1, float("nan"), None) == \
         binding.MUON_ERR_INVALID_ARG
+
+
+def test_closed_plan_refuses_bound_calls(L):
+    """A step bound to a plan reads the plan's handle at call time: once the
+    plan is closed the call raises instead of passing a freed handle on."""
+    plan = binding.MuonPlan.__new__(binding.MuonPlan)
+    plan._h = None
+    with pytest.raises(binding.MuonError) as e:
+        plan._live_handle()
+    assert e.value.status == binding.MUON_ERR_INVALID_ARG
+    plan.close()                         # closing twice is harmless
