@@ -384,11 +384,11 @@ def step_launches(ns_steps: int) -> int:
 def adamw_ema_bind(params: Sequence, grads: Sequence, exp_avgs: Sequence,
                    exp_avg_sqs: Sequence, emas: Sequence, hyper, ema_decay: float,
                    step: int = 1, step_dev=None):
-    """Marshals adamw_ema_batched once and returns `run(step=None,
+    """Marshals adamw_ema_batched once and returns `run(step_now=None,
     stream=None)`.  All tensors fp32 CUDA, contiguous, same numel per index;
     emas[i] may be None.  hyper: an object with lr, beta1, beta2, eps,
     weight_decay.  With step_dev (one-element int32 CUDA tensor) the device
-    counter gives the step; otherwise `step` (or run's argument)."""
+    counter gives the step; otherwise `step`, or run's `step_now`."""
     import torch
     n = len(params)
     if not (len(grads) == len(exp_avgs) == len(exp_avg_sqs) == len(emas) == n):
@@ -459,6 +459,8 @@ def muon_step_batched_noalloc(weights, momenta, grads, hyper, coeffs,
         raise ValueError("one weight, momentum and gradient per matrix")
     mats = (muon_matrix_t * max(n, 1))()
     for i in range(n):
+        if weights[i].dim() != 2:
+            raise ValueError(f"weights[{i}] must be a matrix")
         r, c = (int(v) for v in weights[i].shape)
         _check_tensor(weights[i], torch.float32, (r, c), f"weights[{i}]")
         _check_tensor(momenta[i], torch.float32, (r, c), f"momenta[{i}]")
@@ -476,6 +478,8 @@ def muon_step_batched_noalloc(weights, momenta, grads, hyper, coeffs,
                       float(hyper.weight_decay), float(hyper.eps_row),
                       float(hyper.eps_frob), int(bool(hyper.nesterov)),
                       int(bool(hyper.eq_r)))
+    if any(len(row) != 3 for row in coeffs):
+        raise ValueError("coeffs: one (a, b, c) row per Newton-Schulz step")
     flat = [float(v) for row in coeffs for v in row]
     carr = (c_float * max(len(flat), 1))(*flat)
     _check(lib().muon_step_batched_noalloc(mats, n, ctypes.byref(hp), carr,
