@@ -44,3 +44,28 @@ def test_bench_workload_pair_k_blocks():
     w = wl.workload(6)
     assert bench.ns_issued_flops(w) == 696 * 11 * 5 * PAIR_BLOCK
     assert bench.ns_issued_flops(w) < _dense(w.shapes, 5)
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` times the oracle on the host and prints one
+    JSON line with the contract's keys (small workload, short budget)."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, MUONB200_ORACLE_BUDGET_S="1")
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference",
+                          "--workload", "1", "--steps", "2", "--warmup", "1"],
+                         cwd=root, env=env, capture_output=True, text=True,
+                         timeout=300, check=True).stdout.strip().splitlines()
+    assert len(out) == 1
+    line = json.loads(out[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup",
+                "ms_per_step", "higher_is_better", "scaling", "vs_baseline",
+                "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["steps"] == 2 and line["warmup"] == 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["kind"] == "oracle"
