@@ -114,7 +114,8 @@ def phase_major_makespan(shapes, steps, clusters):
 
 
 @pytest.mark.parametrize("widx,steps,clusters", [(2, 5, 74), (3, 4, 74),
-                                                 (4, 5, 74), (1, 5, 74)])
+                                                 (4, 5, 74), (1, 5, 74),
+                                                 (5, 5, 74)])
 def test_schedule_valid_and_no_worse(exe, widx, steps, clusters):
     shapes = wl.workload(widx).shapes
     items, makespan = run(exe, shapes, steps, clusters)
