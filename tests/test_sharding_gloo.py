@@ -123,6 +123,9 @@ def test_flat_layout_is_owner_ordered_and_aligned():
         assert L.numel() == world * L.seg
 
 
+SHARES = {2: [0.25, 0.75], 4: [0.125, 0.25, 0.25, 0.375]}
+
+
 def _flat_worker(rank, world, port, q):
     import oracle.muon_oracle as mo
     os.environ["MASTER_ADDR"] = "127.0.0.1"
@@ -150,7 +153,8 @@ def _flat_worker(rank, world, port, q):
 
         for step in range(2):
             G_flat = torch.zeros(L.numel(), dtype=torch.float64)
-            share = 0.25 if rank == 0 else 0.75
+            # dyadic shares: the reduce-scatter sums them back to g exactly
+            share = SHARES[world][rank]
             for i, v in enumerate(L.views(G_flat)):
                 g = wl.bf16_bits_to_f32(wl.grad_bits(w, i, step)).astype(np.float64)
                 v.copy_(torch.from_numpy(g * share))
@@ -160,9 +164,9 @@ def _flat_worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_flat_sharded_step_matches_single_process():
+@pytest.mark.parametrize("world", [2, 4])
+def test_flat_sharded_step_matches_single_process(world):
     import oracle.muon_oracle as mo
-    world = 2
     port = _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
