@@ -19,29 +19,16 @@ MuonEq-R, Polar Express 4 steps); PR #1557 "Techniques" (Muon 0.97, LR 0.03).
 
 from __future__ import annotations
 
-import json
 import math
-import os
 from dataclasses import dataclass, field
 from typing import List, Optional, Sequence, Tuple
 
 import numpy as np
 
-REPO_ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-
 # The widely used fixed quintic Muon coefficients.  Not printed on the pages;
 # used as the default "fixed coefficients" input table (the library treats the
 # table purely as input).
 FIXED_QUINTIC = (3.4445, -4.7750, 2.0315)
-
-
-def polar_express_k4() -> List[Tuple[float, float, float]]:
-    """The 4-step greedy minimax table written by
-    tests/golden/make_polar_express.py."""
-    path = os.path.join(REPO_ROOT, "tests", "golden", "polar_express_k4.json")
-    with open(path) as f:
-        doc = json.load(f)
-    return [tuple(r) for r in doc["coeffs"]]
 
 
 @dataclass(frozen=True)
@@ -126,13 +113,18 @@ def gpt11_ema_extras() -> Tuple[List[int], List[str]]:
     return numels, names
 
 
-def _cfg3() -> Workload:
+def _cfg3(ns_coeffs) -> Workload:
+    """The 4-step table is an input (the pages print no coefficients); the
+    tests and the benchmark pass the committed minimax table."""
+    if ns_coeffs is None or len(ns_coeffs) != 4:
+        raise ValueError("the K=4 workload needs its 4-row (a, b, c) table "
+                         "as ns_coeffs")
     numels, names = gpt11_ema_extras()
     return Workload(
         name="11L x 512d GPT, 66 matrices, K=4 Polar-Express table + EMA",
         shapes=_gpt11_shapes(),
         hyper=Hyper(momentum=0.97, lr=0.03, weight_decay=0.105),
-        coeffs=polar_express_k4(), ema_decay=0.9965,
+        coeffs=[tuple(float(v) for v in r) for r in ns_coeffs], ema_decay=0.9965,
         ema_extra_numels=numels, ema_extra_names=names, wid=3)
 
 
@@ -168,10 +160,14 @@ def _cfg_bench() -> Workload:
     return w
 
 
-WORKLOADS = {1: _cfg1, 2: _cfg2, 3: _cfg3, 4: _cfg4, 5: _cfg5, 6: _cfg_bench}
+WORKLOADS = {1: _cfg1, 2: _cfg2, 4: _cfg4, 5: _cfg5, 6: _cfg_bench}
 
 
-def workload(idx: int) -> Workload:
+def workload(idx: int, ns_coeffs=None) -> Workload:
+    """Workload idx (1-6).  Workload 3 runs a 4-step coefficient table that
+    the caller passes as ns_coeffs (rows of (a, b, c))."""
+    if idx == 3:
+        return _cfg3(ns_coeffs)
     return WORKLOADS[idx]()
 
 

@@ -26,7 +26,7 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["minimax_odd_quintic", "polar_express_table"]
+__all__ = ["minimax_odd_quintic", "polar_express_table", "composed_band"]
 
 
 def _solve_reference(xs: np.ndarray) -> tuple[np.ndarray, float]:
@@ -113,3 +113,12 @@ def polar_express_table(steps: int = 4, lo: float = 1e-3, hi: float = 1.0,
         rows.append(coef)
         lo, hi = _image(coef, lo, hi)
     return rows, intervals, design
+
+
+def composed_band(rows, lo: float, hi: float) -> tuple[float, float]:
+    """Exact range of the composed schedule p_K o ... o p_1 over [lo, hi]:
+    each step's exact image (end points and interior critical points) is the
+    next step's domain."""
+    for coef in rows:
+        lo, hi = _image(coef, lo, hi)
+    return lo, hi

@@ -210,6 +210,26 @@ def pin_polar_express_table(o_pe):
     g = np.linspace(lo3, hi3, 400001)
     p = a * g + b * g ** 3 + c * g ** 5
     assert y.min() >= p.min() - 1e-9 and y.max() <= p.max() + 1e-9
+    # the recorded composed band is the range of the scalar chain over the
+    # initial interval (dense sampling, geometric and linear, from below)
+    xs = np.concatenate([np.geomspace(lo0, hi0, 400001), np.linspace(lo0, hi0, 400001)])
+    ys = _scalar_poly_chain(xs, rows)
+    band = doc["band"]
+    assert band[0] <= ys.min() + 1e-12 and ys.max() <= band[1] + 1e-12
+    assert ys.min() - band[0] < 1e-6 and band[1] - ys.max() < 1e-6
+    # the design interval tracks the true lower end: four different steps
+    for i in range(4):
+        for j in range(i + 1, 4):
+            assert np.max(np.abs(np.array(rows[i]) - np.array(rows[j]))) > 1e-3
+    # the plain greedy chain (no margins) equioscillates around 1 on the
+    # whole initial interval: its band is [1 - E, 1 + E], narrower than the
+    # table's margin-widened band
+    plain, _, _ = o_pe.polar_express_table(4, lo0, hi0)
+    yp = _scalar_poly_chain(xs, plain)
+    pb = doc["band_plain_greedy"]
+    assert abs(yp.min() - pb[0]) < 1e-6 and abs(yp.max() - pb[1]) < 1e-6
+    assert abs((pb[0] + pb[1]) - 2.0) < 1e-9
+    assert pb[0] >= band[0] and pb[1] <= band[1]
     # the plain greedy schedule (no margins) is a minimax chain too
     r0, iv0, _ = o_pe.polar_express_table(2, 1e-3, 1.0)
     (a, b, c) = r0[0]

@@ -11,6 +11,7 @@ import pytest
 
 import oracle.muon_oracle as mo
 from gpu_harness import GpuMuon, TOL_STATE, check_step, rel_fro
+import tables
 from muon_optimizer_step_02_b200 import workloads as wl
 
 pytestmark = pytest.mark.gpu
@@ -28,7 +29,7 @@ def test_single_128():
 
 @pytest.mark.parametrize("cfg", [2, 3])
 def test_gpt11_all_matrices(cfg):
-    w = wl.workload(cfg)
+    w = tables.workload(cfg)
     g = GpuMuon(w)
     rep = []
     for step in range(3):
@@ -84,7 +85,7 @@ def _ema_check(w, idx_check):
 
 
 def test_ema_gpt11_all_tensors():
-    w = wl.workload(3)
+    w = tables.workload(3)
     _ema_check(w, set(range(len(w.ema_numels()))))
 
 

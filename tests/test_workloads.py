@@ -2,6 +2,7 @@
 determinism of the generators.  CPU only."""
 import numpy as np
 
+import tables
 from muon_optimizer_step_02_b200 import workloads as wl
 
 
@@ -19,7 +20,7 @@ def test_gpt11_ema_parameter_count():
     """Explicit tensor list of the EMA workload: 66 matrices + 8192x512 +
     4096x512 embeddings + 118 x 512 vectors + 92 scalars = 38,071,388; the
     1-D part is sized to the page's 34,401,372-parameter residual."""
-    w = wl.workload(3)
+    w = tables.workload(3)
     n = w.ema_numels()
     assert len(n) == 66 + 2 + 118 + 92
     assert sum(n) == 38_071_388
@@ -55,6 +56,11 @@ def test_bf16_bits_round_to_nearest_even():
     assert back.tolist() == [1.0, 1.0, 1.0 + 2 ** -6, -2.5]
 
 
-def test_polar_express_table_loads():
-    t = wl.polar_express_k4()
+def test_polar_express_table_is_an_input():
+    t = tables.polar_express_k4()
     assert len(t) == 4 and all(len(r) == 3 for r in t)
+    assert tables.workload(3).coeffs == [tuple(r) for r in t]
+    # the package reads no table itself: workload 3 needs one passed in
+    import pytest
+    with pytest.raises(ValueError):
+        wl.workload(3)
