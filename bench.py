@@ -79,6 +79,16 @@ def recorded_traffic(kernel: str, workload: int):
     return rec.get("dram_bytes_per_launch")
 
 
+def load_workload(idx: int) -> wl.Workload:
+    """Workload idx; the K=4 workload takes the committed 4-step minimax table
+    (tests/golden/polar_express_k4.json, written by an oracle/ script) as its
+    Newton-Schulz input."""
+    if idx != 3:
+        return wl.workload(idx)
+    with open(os.path.join(ROOT, "tests", "golden", "polar_express_k4.json")) as f:
+        return wl.workload(3, json.load(f)["coeffs"])
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -232,7 +242,7 @@ def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     torch.cuda.set_device(local_rank)
-    w = wl.workload(args.workload)
+    w = load_workload(args.workload)
     rep = Workload(w, seed=1337 + rank)
     stream = torch.cuda.current_stream()
     peaks, peak_src = load_peaks()
@@ -260,29 +270,36 @@ def run_ours(args, rank, world, local_rank):
         assert rep.plan.last_error() == 0
     run_step = graph.replay if graph is not None else rep.step
 
-    # ---- timed region: device time with CUDA events on the launching stream
+    # ---- timed region: device time with CUDA events on the launching
+    # stream.  The block of K steps is timed `repeats` times (each bracketed
+    # by a barrier and synchronisations); the median block is reported, and
+    # the clock sampler runs across all of them.
     clocks = ClockSampler(local_rank)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
+    blocks = []
     clocks.start()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(args.steps):
-        run_step()
-    t1.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    for _ in range(args.repeats):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            run_step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        blk = t0.elapsed_time(t1)
+        if world > 1:
+            t = torch.tensor([blk], device="cuda", dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            blk = float(t.item())
+        blocks.append(blk)
     clk = clocks.stop()
-    ms = t0.elapsed_time(t1)
     if rep.plan.last_error() != 0:
         raise RuntimeError("device-side error during the timed region")
-    if world > 1:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = statistics.median(blocks)
     ms_per_step = ms / args.steps
     value = world * args.steps / (ms / 1e3)
 
@@ -404,6 +421,12 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return None
 
+    # ---- the largest workload (24L x 2048d), one GPU only
+    largest = None
+    if world == 1 and not args.no_largest:
+        largest = measure_largest(stream, local_rank, peaks, peak_src,
+                                  args.largest_replays)
+
     # ---- yardstick: the same Newton-Schulz work as torch/cuBLAS GEMMs
     yard_ms = (torch_ns_yardstick(w, stream, max(3, min(args.steps, 20)))
                if not args.no_yardstick else None)
@@ -413,20 +436,28 @@ def run_ours(args, rank, world, local_rank):
     ns_kinds = ("gram", "poly", "apply", "ns")
     dom = max(phase, key=lambda k: phase[k][1])
     launches_dom, ms_dom = phase[dom]
-    sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    # The Newton-Schulz launch is timed alone (about 0.4 ms per launch in a
+    # loop of a few milliseconds), so its peak is the burst bf16 figure.
+    burst = peaks["bf16_tflops"]
     if dom in ns_kinds:
         per_launch = flops[dom]
-        achieved = per_launch / (ms_dom / launches_dom / 1e3) / 1e12
+        dt = ms_dom / launches_dom / 1e3
+        achieved = per_launch / dt / 1e12
         kname = "ns_mega_pair_kernel" if dom == "ns" else dom
+        issued = ns_issued_flops(w) / dt / 1e12 if dom == "ns" else None
         roof = {"kernel": f"{kname} (all {len(w.coeffs)} Newton-Schulz steps)"
                 if dom == "ns" else dom,
                 "bound": "tensor",
-                "achieved": round(achieved, 2), "peak": sustained,
-                "unit": "TFLOP/s", "frac": round(achieved / sustained, 4),
+                "achieved": round(achieved, 2), "peak": burst,
+                "unit": "TFLOP/s", "frac": round(achieved / burst, 4),
+                "issued_tflops": round(issued, 2) if issued else None,
+                "issued_frac": round(issued / burst, 4) if issued else None,
                 "traffic": recorded_traffic(kname, args.workload),
                 "traffic_unit": "bytes per launch (ncu dram read + write)",
                 "flops_per_launch": per_launch,
-                "peak_source": f"{peak_src} sustained bf16"}
+                "flops_count": "dense 4m^2n + 2m^3 per matrix and step; "
+                               "issued = the pair k-blocks the kernel runs",
+                "peak_source": f"{peak_src} burst bf16 (kernel timed per launch)"}
     else:
         per_launch = rep.state_bytes()["prologue"]
         achieved = per_launch / (ms_dom / launches_dom / 1e3) / 1e9
@@ -435,8 +466,6 @@ def run_ours(args, rank, world, local_rank):
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": None, "peak_source": f"{peak_src} HBM copy"}
     ns_ms = sum(phase[k][1] for k in ns_kinds if k in phase) / args.steps
-    ns_flops = flops["ns"]
-    ns_tflops = ns_flops / (ns_ms / 1e3) / 1e12 if ns_ms > 0 else None
     pro_ms = phase["prologue"][1] / max(phase["prologue"][0], 1)
     breakdown = {k: {"launches": v[0], "ms_per_step": round(v[1] / args.steps, 4)}
                  for k, v in phase.items() if v[0] > 0}
@@ -456,23 +485,23 @@ def run_ours(args, rank, world, local_rank):
                          "resident, all of it read or written every step)",
                    "mode": "eager launches" if args.eager
                    else "CUDA graph replay (one graph per step)",
+                   "timing": f"median of {args.repeats} timed blocks of "
+                             f"{args.steps} steps each",
                    "eager_steps_per_s": round(eager_value, 3)},
         "clocks": clk,
         "e2e": {"value": round(e2e_value, 3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4,
                 "how": "all gradients uploaded as one copy from pinned memory on a "
                        "copy stream, double-buffered; each step's status word copied "
-                       "back and checked one step later"},
+                       "back and checked one step later.  Weights, momenta and "
+                       "averages stay resident on the device (an optimizer's state "
+                       "lives where the model does), so the only result read back "
+                       "per step is the 4-byte status word"},
         "gpu_launches": rep.launches_per_step() * args.steps,
         "roofline": roof,
-        "ns": {"tflops": round(ns_tflops, 2) if ns_tflops else None,
-               "frac_of_sustained": round(ns_tflops / sustained, 4)
-               if ns_tflops else None, "ms_per_step": round(ns_ms, 4),
-               "issued_tflops": round(ns_issued_flops(w) / (ns_ms / 1e3) / 1e12, 2)
-               if ns_ms > 0 else None,
-               "issued_flops_per_launch": ns_issued_flops(w)},
-        "prologue_gbs": round(rep.state_bytes()["prologue"] / (pro_ms / 1e3) / 1e9, 1)
-        if pro_ms > 0 else None,
+        "ns": ns_record(ns_ms, flops["ns"], ns_issued_flops(w), burst,
+                        "burst (timed per launch)"),
+        "prologue": prologue_record(pro_ms, w.numel(), peaks["hbm_gbs"]),
         "ema": {"gbs": round(ema_gbs, 1) if ema_gbs else None,
                 "frac": round(ema_gbs / peaks["hbm_gbs"], 4) if ema_gbs else None,
                 "ms": round(ema_ms, 4) if ema_ms else None},
@@ -486,6 +515,8 @@ def run_ours(args, rank, world, local_rank):
             "ns_ms": round(yard_ms, 4),
             "tflops": round(flops["ns"] / (yard_ms / 1e3) / 1e12, 2),
             "fused_speedup": round(yard_ms / ns_ms, 3) if ns_ms > 0 else None}
+    if largest is not None:
+        line["largest"] = largest
     if adamw is not None:
         a_ms, a_params = adamw
         a_gbs = 36 * a_params / (a_ms / 1e3) / 1e9
@@ -494,6 +525,134 @@ def run_ours(args, rank, world, local_rank):
                              "frac": round(a_gbs / peaks["hbm_gbs"], 4),
                              "bytes_per_param": 36}
     return line
+
+
+def ns_record(ns_ms, dense_flops, issued_flops, peak, peak_name):
+    """Newton-Schulz time per step with its dense (4m^2n + 2m^3 per matrix
+    and step) and issued (pair k-blocks run) rates against `peak`."""
+    if not ns_ms or ns_ms <= 0:
+        return None
+    dense = dense_flops / (ns_ms / 1e3) / 1e12
+    issued = issued_flops / (ns_ms / 1e3) / 1e12
+    return {"ms_per_step": round(ns_ms, 4), "tflops": round(dense, 2),
+            "issued_tflops": round(issued, 2), "peak": peak, "peak_kind": peak_name,
+            "frac": round(dense / peak, 4), "issued_frac": round(issued / peak, 4),
+            "dense_flops": dense_flops, "issued_flops": issued_flops}
+
+
+def prologue_record(pro_ms, elems, hbm_gbs):
+    """The prologue's rate counted two ways: the algorithmic 10 B per matrix
+    element of the momentum step (G read 2, M read 4 and written 4), and the
+    12 B it moves (plus the bf16 working copy written)."""
+    if not pro_ms or pro_ms <= 0:
+        return None
+    alg = 10 * elems / (pro_ms / 1e3) / 1e9
+    moved = 12 * elems / (pro_ms / 1e3) / 1e9
+    return {"ms": round(pro_ms, 4), "gbs": round(alg, 1), "frac": round(alg / hbm_gbs, 4),
+            "bytes_per_elem": 10, "moved_gbs": round(moved, 1),
+            "moved_frac": round(moved / hbm_gbs, 4), "moved_bytes_per_elem": 12}
+
+
+def measure_largest(stream, local_rank, peaks, peak_src, replays):
+    """The 24L x 2048d set (144 matrices, K=5 fixed quintic) plus the EMA over
+    its 1.14 G parameters, one CUDA graph per step replayed `replays` times
+    (about a second of dense tensor work, so the sustained bf16 peak
+    applies), with its own clock record; then a few eager steps for the
+    per-kernel split.  Inputs are drawn on the device from a seeded generator
+    (same distributions as the 11L set's host-drawn inputs)."""
+    import torch
+    from muon_optimizer_step_02_b200 import binding as B
+    w = wl.workload(5)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1337)
+    plan = B.MuonPlan(w.shapes, max_ns_steps=len(w.coeffs))
+    ws = plan.alloc_workspace()
+    W = [torch.randn(r, c, device="cuda", generator=gen).mul_(w.weight_std)
+         for r, c in w.shapes]
+    M = [torch.zeros_like(x) for x in W]
+    G = [torch.randn(r, c, device="cuda", generator=gen).mul_(w.grad_std)
+         .to(torch.bfloat16) for r, c in w.shapes]
+    extra = [torch.randn(n, device="cuda", generator=gen).mul_(0.02)
+             for n in w.ema_extra_numels]
+    E = [x.clone().view(-1) for x in W] + [x.clone() for x in extra]
+    P = [x.view(-1) for x in W] + extra
+    muon = plan.bind(W, M, G, w.hyper, w.coeffs, ws, update_scales=wl.update_scales(w))
+    ema = B.ema_bind(E, P, w.ema_decay)
+
+    def step():
+        muon()
+        ema()
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    if plan.last_error() != 0:
+        raise RuntimeError("device-side error in the 24L warm-up")
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            step()
+    stream.wait_stream(side)
+    graph.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(replays):
+        graph.replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1) / replays
+    del graph
+    # per-kernel split from eager steps (plan events; the EMA on own events)
+    plan.set_timing(True)
+    plan.timing_read()
+    n_eager = 3
+    e_ms = 0.0
+    for _ in range(n_eager):
+        muon()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        ema()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        e_ms += a0.elapsed_time(a1)
+    phase = plan.timing_read()
+    plan.set_timing(False)
+    if plan.last_error() != 0:
+        raise RuntimeError("device-side error in the 24L timing")
+    ns_ms = phase["ns"][1] / max(phase["ns"][0], 1)
+    pro_ms = phase["prologue"][1] / max(phase["prologue"][0], 1)
+    ema_ms = e_ms / n_eager
+    ema_params = sum(w.ema_numels())
+    ema_gbs = 12 * ema_params / (ema_ms / 1e3) / 1e9
+    dense = sum(2 * min(r, c) ** 2 * max(r, c) * 2 + 2 * min(r, c) ** 3
+                for r, c in w.shapes) * len(w.coeffs)
+    sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    rec = {"workload": w.name, "n_mats": w.n_mats, "matrix_params": w.numel(),
+           "ema_params": ema_params, "ns_steps": len(w.coeffs),
+           "data": "synthetic, drawn on the device (torch.Generator seed 1337): "
+                   "W ~ N(0, 0.02^2), G ~ N(0, 1e-3^2) in bf16, E = W, M = 0",
+           "steps_per_s": round(1e3 / ms, 3), "ms_per_step": round(ms, 3),
+           "replays": replays, "mode": "CUDA graph replay (one graph per step)",
+           "clocks": clk,
+           "ns": ns_record(ns_ms, dense, ns_issued_flops(w), sustained,
+                           f"{peak_src} sustained (a ~40 ms kernel in a "
+                           "seconds-long loop)"),
+           "prologue": prologue_record(pro_ms, w.numel(), peaks["hbm_gbs"]),
+           "ema": {"ms": round(ema_ms, 4), "gbs": round(ema_gbs, 1),
+                   "frac": round(ema_gbs / peaks["hbm_gbs"], 4), "bytes_per_param": 12},
+           "per_kernel_from": f"{n_eager} eager steps, CUDA events on the stream"}
+    plan.close()
+    del W, M, G, E, P, extra, ws
+    torch.cuda.empty_cache()
+    return rec
 
 
 def adamw_ema_measure(w, stream, reps):
@@ -657,7 +816,7 @@ def oracle_sample(w: wl.Workload, budget_s: float, seed: int = 1337):
 def run_reference(args, rank):
     if rank != 0:
         return None
-    w = wl.workload(args.workload)
+    w = load_workload(args.workload)
     budget = float(os.environ.get("MUONB200_ORACLE_BUDGET_S", "20"))
     times, desc, threads = [], "", os.cpu_count()
     for _ in range(args.warmup):
@@ -692,6 +851,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-yardstick", action="store_true",
                     help="skip timing the same Newton-Schulz work as torch/cuBLAS GEMMs")
+    ap.add_argument("--repeats", type=int, default=5,
+                    help="timed blocks of --steps steps; the median is reported")
+    ap.add_argument("--no-largest", action="store_true",
+                    help="skip the 24L x 2048d sub-record")
+    ap.add_argument("--largest-replays", type=int, default=20)
     ap.add_argument("--eager", action="store_true",
                     help="time eager launches instead of one CUDA graph per step")
     args = ap.parse_args()
@@ -724,7 +888,7 @@ def main():
         return
     if not args.no_cpu_baseline:
         budget = float(os.environ.get("MUONB200_ORACLE_BUDGET_S", "15"))
-        s, desc, threads = oracle_sample(wl.workload(args.workload), budget)
+        s, desc, threads = oracle_sample(load_workload(args.workload), budget)
         line["cpu_baseline"] = {"value": round(1.0 / s, 6), "unit": UNIT,
                                 "cores": threads, "kind": "oracle",
                                 "sample": desc}
@@ -733,7 +897,7 @@ def main():
         try:
             from threadpoolctl import threadpool_limits
             with threadpool_limits(limits=1):
-                s1, desc1, _ = oracle_sample(wl.workload(args.workload), budget / 3)
+                s1, desc1, _ = oracle_sample(load_workload(args.workload), budget / 3)
             line["cpu_baseline"]["one_thread"] = {"value": round(1.0 / s1, 6),
                                                   "unit": UNIT, "sample": desc1}
         except ImportError:

@@ -42,8 +42,9 @@
  *    muon_get_last_error (synchronises `stream`), muon_plan_timing_read and
  *    muon_plan_destroy (synchronise the device).
  *  - Argument, shape and alignment errors are detected on the host and
- *    returned before anything is enqueued.  Launch failures return
- *    MUON_ERR_CUDA.  A device-side wait that exceeds its time limit (about one
+ *    returned before anything is enqueued.  A refused launch returns
+ *    MUON_ERR_CUDA and nothing after it is enqueued (the call's earlier
+ *    launches have run).  A device-side wait that exceeds its time limit (about one
  *    second) makes the kernel record an error word, drain its own copies and
  *    return; muon_get_last_error reports it as MUON_ERR_TIMEOUT.
  */
@@ -223,6 +224,17 @@ muon_status_t adamw_ema_batched(const adamw_tensor_t *tensors, int32_t n_tensors
                                 int32_t *step_dev, float ema_decay,
                                 muon_stream_t stream);
 
+/* dst[i] = src[i] rounded to bf16 (nearest, ties to even), i < n: one pass
+ * over device memory (src fp32, 4-byte aligned; dst bf16 bit patterns,
+ * 2-byte aligned; 16-byte aligned arrays take the vectorised path).  For a
+ * gradient reduced in fp32 across data-parallel ranks (PR #1893, table
+ * "Architecture and training stack", row "Train context": 8-way training)
+ * and handed to the Muon step, which reads bf16 gradients.  Asynchronous on
+ * `stream`; MUON_ERR_INVALID_ARG for n < 0 or a NULL array with n > 0,
+ * MUON_ERR_ALIGNMENT for misaligned arrays. */
+muon_status_t muon_f32_to_bf16(uint16_t *dst, const float *src, int64_t n,
+                               muon_stream_t stream);
+
 /* Synchronises `stream`, reads and clears the plan's device error word.
  * Returns MUON_ERR_TIMEOUT if a kernel gave up on a bounded wait since the
  * last call, MUON_ERR_CUDA on a CUDA error, MUON_OK otherwise. */
@@ -288,6 +300,11 @@ muon_status_t muon_plan_set_fault(muon_plan_t *plan, int32_t fault);
 /* ABI version (major * 100 + minor). */
 int32_t muon_abi_version(void);
 
+/* Number of device allocations (cudaMalloc) this library has made in the
+ * process so far: one per muon_plan_create, none in any other call.  Lets a
+ * caller check that a code path allocated nothing. */
+int64_t muon_device_allocation_count(void);
+
 /* ---- One batched step without any device allocation ----------------------
  * The pages have no counterpart to this call.  It is for callers that cannot
  * allocate device memory: a framework that owns every device allocation
@@ -314,8 +331,11 @@ int32_t muon_abi_version(void);
  * the error word with cudaMemsetAsync, and calls no cudaMalloc, cudaFree or
  * other allocating routine.  All calls share the one array: calls that overlap
  * on the GPU (different streams, or different host threads without ordering)
- * race on it; order them on one stream.  Device-side wait timeouts in this
- * path set the array's error word but are not reported back to the host. */
+ * race on it; order them on one stream.  A device-side wait that runs out
+ * (the step then stops early and leaves W and the momentum partly updated)
+ * sets the array's error word, which each call clears at its start and
+ * muon_noalloc_error_async reads back.  A refused launch returns
+ * MUON_ERR_CUDA at once and enqueues nothing after it. */
 #define MUON_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 #define MUON_NOALLOC_MAX_MATS 64
 muon_status_t muon_step_batched_noalloc(const muon_matrix_t *mats,
@@ -324,6 +344,22 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t *mats,
                                         const float *ns_coeffs,
                                         int32_t ns_steps,
                                         muon_stream_t stream);
+
+/* Enqueues on `stream` a copy of the allocation-free path's error word (of
+ * the current device) into *host_word (host memory; pinned for the copy to
+ * be asynchronous), without synchronising and without allocating.  Read it
+ * after the stream has passed this point: non-zero means a kernel of the last
+ * muon_step_batched_noalloc call enqueued before it gave up on a bounded wait
+ * (that step is incomplete).  Returns MUON_ERR_INVALID_ARG for a NULL
+ * host_word, MUON_ERR_CUDA if the copy cannot be enqueued.  The pages have
+ * no counterpart to this call either. */
+muon_status_t muon_noalloc_error_async(int32_t *host_word, muon_stream_t stream);
+
+/* Test hook of the allocation-free path, process-wide: the faults of
+ * muon_plan_set_fault (1: a bounded wait runs out; 2: the tensor-core
+ * kernel's launch is refused) for later muon_step_batched_noalloc calls; 0
+ * turns it off. */
+muon_status_t muon_noalloc_set_fault(int32_t fault);
 
 #ifdef __cplusplus
 }

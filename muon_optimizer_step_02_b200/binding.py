@@ -139,6 +139,14 @@ def lib():
                                             POINTER(c_float), c_int32,
                                             c_void_p]
     L.muon_step_batched_noalloc.restype = c_int32
+    L.muon_noalloc_error_async.argtypes = [c_void_p, c_void_p]
+    L.muon_noalloc_error_async.restype = c_int32
+    L.muon_noalloc_set_fault.argtypes = [c_int32]
+    L.muon_noalloc_set_fault.restype = c_int32
+    L.muon_f32_to_bf16.argtypes = [c_void_p, c_void_p, c_int64, c_void_p]
+    L.muon_f32_to_bf16.restype = c_int32
+    L.muon_device_allocation_count.argtypes = []
+    L.muon_device_allocation_count.restype = c_int64
     _lib = L
     return L
 
@@ -486,3 +494,40 @@ def muon_step_batched_noalloc(weights, momenta, grads, hyper, coeffs,
                                            len(flat) // 3,
                                            _stream_handle(stream)),
            "muon_step_batched_noalloc")
+
+
+def noalloc_error_async(host_word, stream=None):
+    """Enqueues a copy of the allocation-free path's error word into
+    `host_word` (a one-element int32 CPU tensor, pinned for the copy to be
+    asynchronous); non-zero once the stream has passed this point means the
+    last muon_step_batched_noalloc call gave up on a bounded wait."""
+    import torch
+    if host_word.dtype != torch.int32 or host_word.device.type != "cpu" or \
+            host_word.numel() < 1:
+        raise ValueError("host_word must be an int32 CPU tensor")
+    _check(lib().muon_noalloc_error_async(host_word.data_ptr(),
+                                          _stream_handle(stream)),
+           "muon_noalloc_error_async")
+
+
+def noalloc_set_fault(fault: int):
+    """Test hook of the allocation-free path (see muon_plan_set_fault)."""
+    _check(lib().muon_noalloc_set_fault(int(fault)), "muon_noalloc_set_fault")
+
+
+def device_allocation_count() -> int:
+    """Device allocations the library has made in this process so far."""
+    return int(lib().muon_device_allocation_count())
+
+
+def f32_to_bf16(dst, src, stream=None):
+    """dst (bf16 CUDA tensor) <- src (fp32 CUDA tensor, same numel) rounded to
+    nearest even, by the library's conversion kernel."""
+    import torch
+    if not (src.is_cuda and dst.is_cuda) or src.dtype != torch.float32 or \
+            dst.dtype != torch.bfloat16 or src.numel() != dst.numel() or \
+            not (src.is_contiguous() and dst.is_contiguous()):
+        raise ValueError("f32_to_bf16: contiguous fp32 src and bf16 dst CUDA "
+                         "tensors of one size")
+    _check(lib().muon_f32_to_bf16(dst.data_ptr(), src.data_ptr(), src.numel(),
+                                  _stream_handle(stream)), "muon_f32_to_bf16")

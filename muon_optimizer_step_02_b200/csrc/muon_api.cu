@@ -13,6 +13,7 @@
 #include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -24,6 +25,7 @@
 
 
 #include "k_adamw_ema.cuh"
+#include "k_convert.cuh"
 #include "k_ema.cuh"
 #include "k_ns_mega.cuh"
 #include "k_prologue.cuh"
@@ -41,6 +43,16 @@ constexpr int kTimingSlots = 64;
 constexpr size_t kProSmemCap = 48 * 1024;   // staging of the transposed write
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Every device allocation of the library goes through dev_alloc, which counts
+// successful ones (muon_device_allocation_count).
+std::atomic<long long> g_device_allocations{0};
+
+cudaError_t dev_alloc(void** p, size_t bytes) {
+  const cudaError_t e = cudaMalloc(p, bytes);
+  if (e == cudaSuccess) g_device_allocations.fetch_add(1, std::memory_order_relaxed);
+  return e;
+}
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
@@ -399,24 +411,42 @@ bool fill_caller_fields(MatDev& d, const muon_matrix_t& mt) {
   return true;
 }
 
-bool set_kernel_attributes(size_t pro_smem, size_t pro_smem_one) {
-  if (cudaFuncSetAttribute(ns_mega_pair_kernel,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kMegaSmemBytes)) != cudaSuccess)
+// The dynamic shared memory limit of a kernel (cudaFuncAttributeMax-
+// DynamicSharedMemorySize) is a per-device, process-wide setting.  Plans of
+// different shapes need different prologue staging sizes, so the limit is
+// only ever raised: each kernel keeps, per device, the largest value set so
+// far (under a mutex), and a plan needing less leaves it alone.  Lowering it
+// would make the launches of an earlier plan that needs more fail.
+constexpr int kMaxDevices = 64;
+struct SmemLimits {
+  size_t ns = 0, pro_two = 0, pro_one = 0;
+};
+std::mutex g_smem_mutex;
+SmemLimits g_smem_limits[kMaxDevices];
+
+bool raise_smem_limit(const void* fn, size_t& cur, size_t want) {
+  if (want <= cur) return true;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(want)) != cudaSuccess)
     return false;
-  // (set whenever there is dynamic shared memory: static plus dynamic above
-  // 48 KB needs the opt-in even when the dynamic part alone is below it)
-  if (pro_smem > 0 &&
-      cudaFuncSetAttribute(muon_prologue_kernel<false>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(pro_smem)) != cudaSuccess)
-    return false;
-  if (pro_smem_one > 0 &&
-      cudaFuncSetAttribute(muon_prologue_kernel<true>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(pro_smem_one)) != cudaSuccess)
-    return false;
+  cur = want;
   return true;
+}
+
+// (a limit is set whenever there is dynamic shared memory: static plus
+// dynamic above 48 KB needs the opt-in even when the dynamic part alone is
+// below it)
+bool set_kernel_attributes(size_t pro_smem, size_t pro_smem_one) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(g_smem_mutex);
+  SmemLimits& lim = g_smem_limits[dev];
+  return raise_smem_limit(reinterpret_cast<const void*>(ns_mega_pair_kernel), lim.ns,
+                          kMegaSmemBytes) &&
+         raise_smem_limit(reinterpret_cast<const void*>(muon_prologue_kernel<false>),
+                          lim.pro_two, pro_smem) &&
+         raise_smem_limit(reinterpret_cast<const void*>(muon_prologue_kernel<true>),
+                          lim.pro_one, pro_smem_one);
 }
 
 cudaLaunchConfig_t pair_launch_config(int clusters, cudaStream_t st,
@@ -460,8 +490,11 @@ void fill_sched_matrix(SchedMatrix& s, const Geom& g) {
 }
 
 // prologue (which also zeroes the step's counters) -> Frobenius scale ->
-// Newton-Schulz (or the finisher for 0 steps).
-void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
+// Newton-Schulz (or the finisher for 0 steps).  Each launch is checked as it
+// is made: if the runtime refuses one, nothing after it is enqueued (a later
+// kernel would otherwise run on partials and counters the refused one never
+// wrote) and MUON_ERR_CUDA is returned; the launches before it have run.
+muon_status_t enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
                   const muon_schedule_t* sched, int32_t* step_dev,
                   const float* ns_coeffs, int32_t ns_steps, const StepScratch& sc,
                   int fault, bool fresh, cudaStream_t st, Recorder* rec) {
@@ -488,31 +521,38 @@ void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
     lr_dev = sc.lr_slot;
   }
   int32_t* done = sc.counters;
+  auto launched = [] { return cudaGetLastError() == cudaSuccess; };
   nvtxRangePushA("muon.prologue");
   if (t.n_one > 0)
     muon_prologue_kernel<true><<<static_cast<unsigned>(t.pro_grid[0]), kProThreads,
                                  t.pro_smem_one, st>>>(t.mats, t.items, t.n_one, hd,
                                                        sc.partials, sc.counters,
                                                        sc.n_counters, t.pro_prefetch);
-  if (t.n_items > t.n_one)
+  bool ok = launched();
+  if (ok && t.n_items > t.n_one) {
     muon_prologue_kernel<false><<<static_cast<unsigned>(t.pro_grid[1]), kProThreads,
                                   t.pro_smem, st>>>(
         t.mats, t.items + t.n_one, t.n_items - t.n_one, hd, sc.partials, sc.counters,
         sc.n_counters, 0);
+    ok = launched();
+  }
   nvtxRangePop();
+  if (!ok) return MUON_ERR_CUDA;
   if (rec) rec->after(MUON_KIND_PROLOGUE);
   nvtxRangePushA("muon.frobenius_scale");
   muon_frob_scale_kernel<<<static_cast<unsigned>((sc.n_mats + 7) / 8), 256, 0, st>>>(
       t.mats, sc.n_mats, sc.partials, hd, sc.mat_scale);
   nvtxRangePop();
+  if (!launched()) return MUON_ERR_CUDA;
   if (rec) rec->after(MUON_KIND_SCALE);
 
   if (ns_steps == 0) {
     muon_final_noiter_kernel<<<static_cast<unsigned>(t.n_items), kProThreads, 0,
                                st>>>(t.mats, t.items, sc.mat_scale, h.lr, lr_dev,
                                      h.weight_decay);
+    if (!launched()) return MUON_ERR_CUDA;
     if (rec) rec->after(MUON_KIND_FINAL);
-    return;
+    return MUON_OK;
   }
   MegaParams p{};
   p.mats = t.mats;
@@ -539,16 +579,23 @@ void enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
   // so that the runtime refuses the launch (no kernel runs)
   if (fault == 2) cfg.dynamicSmemBytes = kMegaSmemBytes + 64 * 1024;
   nvtxRangePushA("muon.newton_schulz");
-  cudaLaunchKernelEx(&cfg, ns_mega_pair_kernel, p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, ns_mega_pair_kernel, p);
   nvtxRangePop();
+  cudaGetLastError();
+  if (e != cudaSuccess) return MUON_ERR_CUDA;
   if (rec) rec->after(MUON_KIND_NS);
+  return MUON_OK;
 }
 
 }  // namespace
 
 extern "C" {
 
-int32_t muon_abi_version(void) { return 100; }
+int32_t muon_abi_version(void) { return 101; }
+
+int64_t muon_device_allocation_count(void) {
+  return g_device_allocations.load(std::memory_order_relaxed);
+}
 
 const char* muon_status_string(muon_status_t s) {
   switch (s) {
@@ -669,7 +716,7 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
       !set_kernel_attributes(plan->pro_smem, plan->pro_smem_one) ||
       (plan->pro_grid[0] = prologue_grid<true>(plan->n_one, plan->pro_smem_one)) < 0 ||
       (plan->pro_grid[1] = prologue_grid<false>(n_two, plan->pro_smem)) < 0 ||
-      cudaMalloc(&plan->d_block, t_off) != cudaSuccess) {
+      dev_alloc(&plan->d_block, t_off) != cudaSuccess) {
     cudaGetLastError();
     delete plan;
     return MUON_ERR_CUDA;
@@ -692,7 +739,7 @@ muon_status_t muon_plan_create(const int32_t* rows, const int32_t* cols,
   plan->h_mats.resize(n_mats);
   plan->sched.resize(plan->sched_cap);
   plan->sgroups.resize(static_cast<size_t>(n_mats) * std::max(max_ns_steps, 1) * 3);
-  plan->sorder.resize(n_mats);
+  plan->sorder.resize(2 * static_cast<size_t>(n_mats) + 1);
   plan->scl.resize(plan->max_clusters);
   *out = plan;
   return MUON_OK;
@@ -835,7 +882,8 @@ muon_status_t step_impl(muon_plan_t* plan, const muon_matrix_t* mats,
   }
   if (resched) {
     const long long n = build_schedule(plan->smats.data(), plan->n_mats, ns_steps,
-                                       plan->max_clusters, plan->sched.data(),
+                                       plan->max_clusters, default_policy(),
+                                       plan->sched.data(),
                                        plan->sched_cap, plan->sgroups.data(),
                                        plan->sorder.data(), plan->scl.data());
     if (n < 0) return MUON_ERR_UNSUPPORTED;
@@ -859,9 +907,11 @@ muon_status_t step_impl(muon_plan_t* plan, const muon_matrix_t* mats,
                  counters_for(plan->n_mats, ns_steps), plan->n_mats,
                  reinterpret_cast<float*>(ws + plan->lr_slot_off)};
   Recorder rec(plan, st);
-  enqueue_step(t, *hyper, sched, step_dev, ns_coeffs, ns_steps, sc, plan->fault, changed,
-               st, plan->timing ? &rec : nullptr);
+  const muon_status_t es = enqueue_step(t, *hyper, sched, step_dev, ns_coeffs, ns_steps,
+                                        sc, plan->fault, changed, st,
+                                        plan->timing ? &rec : nullptr);
   rec.finish();
+  if (es != MUON_OK) return es;
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
 }
@@ -946,6 +996,32 @@ muon_status_t ema_update_batched(float* const* ema, const float* const* params,
     ema_update_kernel<<<grid, kEmaThreads, 0, st>>>(p);
     nvtxRangePop();
   }
+  if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
+  return MUON_OK;
+}
+
+muon_status_t muon_f32_to_bf16(uint16_t* dst, const float* src, int64_t n,
+                               muon_stream_t stream) {
+  if (n < 0) return MUON_ERR_INVALID_ARG;
+  if (n == 0) return MUON_OK;
+  if (!dst || !src) return MUON_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(dst) & 1u) || (reinterpret_cast<uintptr_t>(src) & 3u))
+    return MUON_ERR_ALIGNMENT;
+  const int vec = ((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src)) &
+                   15u) == 0 ? 1 : 0;
+  int sms = 148;
+  {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MUON_ERR_CUDA;
+  }
+  const long long per_thread = vec ? 8 : 1;
+  const long long want = (n / per_thread + kCvtThreads - 1) / kCvtThreads;
+  const unsigned grid =
+      static_cast<unsigned>(std::max(1ll, std::min<long long>(want, 8ll * sms)));
+  f32_to_bf16_kernel<<<grid, kCvtThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      dst, src, n, vec);
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
 }
@@ -1050,8 +1126,34 @@ ProItem g_na_items[kNoAllocMaxItems];
 SchedMatrix g_na_smats[MUON_NOALLOC_MAX_MATS];
 SchedItem g_na_sched[kNoAllocMaxSched];
 SchedGroup g_na_groups[kNoAllocMaxGroups];
-int g_na_order[MUON_NOALLOC_MAX_MATS];
+int g_na_order[2 * MUON_NOALLOC_MAX_MATS + 1];
 double g_na_cltime[kNoAllocMaxClusters];
+
+// Test hook of the allocation-free path (muon_noalloc_set_fault).
+int g_noalloc_fault = 0;
+
+// Set-up of the current device, once per device, with g_noalloc_mutex held:
+// the device address of g_noalloc_scratch (cudaGetSymbolAddress, with this
+// device current) and the cluster count of the tensor-core kernel.  *dev
+// receives the current device.
+muon_status_t noalloc_setup(int& dev) {
+  if (cudaGetDevice(&dev) != cudaSuccess) return MUON_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return MUON_ERR_UNSUPPORTED;
+  if (g_noalloc_dev_ptr[dev]) return MUON_OK;
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+    cudaGetLastError();
+    return MUON_ERR_CUDA;
+  }
+  const int clusters = query_max_clusters();
+  if (clusters <= 0 || clusters > kNoAllocMaxClusters) {
+    cudaGetLastError();
+    return MUON_ERR_CUDA;
+  }
+  g_noalloc_clusters[dev] = clusters;
+  g_noalloc_dev_ptr[dev] = ptr;
+  return MUON_OK;
+}
 
 }  // namespace
 
@@ -1104,26 +1206,13 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
 
   // Device address of the array on the current device (once per device).
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MUON_ERR_CUDA;
-  if (dev < 0 || dev >= kNoAllocMaxDevices) return MUON_ERR_UNSUPPORTED;
-  if (!g_noalloc_dev_ptr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
-      cudaGetLastError();
-      return MUON_ERR_CUDA;
-    }
-    const int clusters = query_max_clusters();
-    if (clusters <= 0 || clusters > kNoAllocMaxClusters) {
-      cudaGetLastError();
-      return MUON_ERR_CUDA;
-    }
-    g_noalloc_clusters[dev] = clusters;
-    g_noalloc_dev_ptr[dev] = ptr;
-  }
+  vs = noalloc_setup(dev);
+  if (vs != MUON_OK) return vs;
   const int clusters = g_noalloc_clusters[dev];
   long long n_sched = 0;
   if (ns_steps > 0) {
-    n_sched = build_schedule(g_na_smats, n_mats, ns_steps, clusters, g_na_sched,
+    n_sched = build_schedule(g_na_smats, n_mats, ns_steps, clusters, default_policy(),
+                             g_na_sched,
                              kNoAllocMaxSched, g_na_groups, g_na_order, g_na_cltime);
     if (n_sched < 0) return MUON_ERR_UNSUPPORTED;
   }
@@ -1180,8 +1269,33 @@ muon_status_t muon_step_batched_noalloc(const muon_matrix_t* mats,
                  reinterpret_cast<float*>(ws + scale_off),
                  reinterpret_cast<int32_t*>(ws + counter_off), n_counters, n_mats,
                  nullptr};
-  enqueue_step(t, *hyper, nullptr, nullptr, ns_coeffs, ns_steps, sc, 0, true, st, nullptr);
+  const muon_status_t es = enqueue_step(t, *hyper, nullptr, nullptr, ns_coeffs, ns_steps,
+                                        sc, g_noalloc_fault, true, st, nullptr);
+  if (es != MUON_OK) return es;
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
+  return MUON_OK;
+}
+
+muon_status_t muon_noalloc_error_async(int32_t* host_word, muon_stream_t stream) {
+  if (!host_word) return MUON_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  int dev = 0;
+  const muon_status_t vs = noalloc_setup(dev);
+  if (vs != MUON_OK) return vs;
+  // word 0 of the array; the next allocation-free call clears it
+  if (cudaMemcpyAsync(host_word, g_noalloc_dev_ptr[dev], sizeof(int32_t),
+                      cudaMemcpyDeviceToHost,
+                      static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return MUON_ERR_CUDA;
+  }
+  return MUON_OK;
+}
+
+muon_status_t muon_noalloc_set_fault(int32_t fault) {
+  if (fault < 0 || fault > 2) return MUON_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  g_noalloc_fault = fault;
   return MUON_OK;
 }
 

@@ -3,13 +3,19 @@
 Every matrix of a Muon step is an independent unit of work, so a model's
 matrices can be split across ranks: each rank steps the matrices it owns and
 the updated weights are then shared.  This module holds the parts of that
-which need no GPU: the assignment of matrices to ranks (longest-processing-
-time first on the step's FLOP count) and two exchange patterns, written
-against torch.distributed so that they run on NCCL (GPUs) and on gloo (CPU
-tests) alike: per-matrix reduce and broadcast (`sharded_step`), and flat
-owner-ordered buffers with one reduce-scatter of the gradients, momentum kept
-only by the owner, and one all-gather of the weights (`ShardLayout`,
-`sharded_step_flat`).
+which need no GPU, written against torch.distributed so that they run on
+NCCL (GPUs) and on gloo (CPU tests) alike:
+
+* the assignment of matrices to ranks (longest-processing-time first on the
+  step's cost);
+* `ShardLayout` / `sharded_step_flat`: flat owner-ordered buffers, one
+  reduce-scatter of the gradients into each owner's segment, the owners'
+  steps (momentum kept by the owner only), one all-gather of the weights;
+* `BucketedLayout` / `sharded_step_bucketed`: the same over buckets of
+  consecutive matrices, with the reduce-scatter of later buckets overlapping
+  the step of earlier ones and each bucket's all-gather overlapping the
+  steps after it (a communication stream beside the compute stream), and an
+  option to reduce the gradients in fp32.
 
 Context: PR #1893 "Record: L_ParallelResiduals_UNetSkips_DepthRecur_Muon_
 1.0901", table "Architecture and training stack", row "Train context"
@@ -20,7 +26,8 @@ Context: PR #1893 "Record: L_ParallelResiduals_UNetSkips_DepthRecur_Muon_
 from __future__ import annotations
 
 import heapq
-from typing import Callable, List, Sequence, Tuple
+from contextlib import nullcontext
+from typing import Callable, List, Optional, Sequence, Tuple
 
 
 def matrix_cost(rows: int, cols: int, ns_steps: int) -> float:
@@ -56,27 +63,6 @@ def rank_loads(shapes, owner, world, ns_steps=5) -> List[float]:
     for (r, c), o in zip(shapes, owner):
         loads[o] += matrix_cost(r, c, ns_steps)
     return loads
-
-
-def sharded_step(W, M, G_local, owner, rank, step_fn: Callable, group=None):
-    """One data-parallel Muon step with matrix ownership.
-
-    W, M, G_local: per-matrix tensors on this rank (W replicated, M only
-    meaningful on the owner, G_local this rank's gradient contribution).
-      1. every gradient is summed onto its owner (reduce to owner);
-      2. each rank steps the matrices it owns: step_fn(indices) updates
-         W[i] and M[i] in place for i in indices;
-      3. the owner broadcasts each updated weight to every rank.
-    Every rank issues the same collectives in the same order."""
-    import torch.distributed as dist
-    for i, o in enumerate(owner):
-        dist.reduce(G_local[i], dst=o, op=dist.ReduceOp.SUM, group=group)
-    mine = [i for i, o in enumerate(owner) if o == rank]
-    if mine:
-        step_fn(mine)
-    for i, o in enumerate(owner):
-        dist.broadcast(W[i], src=o, group=group)
-    return mine
 
 
 class ShardLayout:
@@ -152,6 +138,131 @@ def sharded_step_flat(layout: ShardLayout, W_flat, M_seg, G_flat, G_seg, rank,
         step_fn(layout.local_views(own, rank), layout.local_views(M_seg, rank),
                 layout.local_views(G_seg, rank))
     dist.all_gather_into_tensor(W_flat, own.clone(), group=group)
+
+
+class BucketedLayout:
+    """The matrices split into `n_buckets` buckets of consecutive plan entries
+    of about equal cost (so that each bucket's step takes about as long), each
+    bucket laid out by its own `ShardLayout` (ownership balanced inside the
+    bucket).  `buckets[b]` lists bucket b's matrices (global indices);
+    `layouts[b]` indexes them 0 .. len(buckets[b]) - 1."""
+
+    def __init__(self, shapes: Sequence[Tuple[int, int]], world: int, n_buckets: int,
+                 ns_steps: int = 5, align: int = 8):
+        self.shapes = [(int(r), int(c)) for r, c in shapes]
+        self.world = world
+        n = len(self.shapes)
+        if not 1 <= n_buckets <= max(n, 1):
+            raise ValueError("need 1 <= n_buckets <= number of matrices")
+        cost = [matrix_cost(r, c, ns_steps) for r, c in self.shapes]
+        total = sum(cost)
+        self.buckets: List[List[int]] = []
+        cur, acc = [], 0.0
+        for i in range(n):
+            cur.append(i)
+            acc += cost[i]
+            left_mats = n - i - 1
+            left_buckets = n_buckets - len(self.buckets) - 1
+            # close the bucket at its share of the cost, keeping at least one
+            # matrix for every bucket still to come
+            if left_buckets > 0 and (acc >= total * (len(self.buckets) + 1) / n_buckets
+                                     or left_mats == left_buckets):
+                self.buckets.append(cur)
+                cur = []
+        self.buckets.append(cur)
+        self.layouts = [ShardLayout([self.shapes[i] for i in bk], world, ns_steps, align)
+                        for bk in self.buckets]
+
+
+class BucketBuffers:
+    """One bucket's buffers on one rank (all flat, 1-D):
+      W_flat  world * seg  weights (replicated after the all-gather);
+      M_seg   seg          momentum of the matrices this rank owns;
+      G_flat  world * seg  this rank's gradient contribution (bf16, or fp32 to
+                           reduce in fp32);
+      G_seg   seg          the summed gradients of this rank's matrices, in
+                           G_flat's dtype;
+      G_step  seg          the gradients the step reads: G_seg itself when the
+                           reduction is in the step's dtype, else a bf16 buffer
+                           that `to_step_dtype` fills from G_seg."""
+
+    def __init__(self, W_flat, M_seg, G_flat, G_seg, G_step=None):
+        self.W_flat, self.M_seg, self.G_flat, self.G_seg = W_flat, M_seg, G_flat, G_seg
+        self.G_step = G_seg if G_step is None else G_step
+
+    @classmethod
+    def allocate(cls, layout: ShardLayout, weight_dtype, grad_dtype, step_grad_dtype,
+                 device=None):
+        import torch
+        W = torch.zeros(layout.numel(), dtype=weight_dtype, device=device)
+        M = torch.zeros(layout.seg, dtype=weight_dtype, device=device)
+        Gf = torch.zeros(layout.numel(), dtype=grad_dtype, device=device)
+        Gs = torch.zeros(layout.seg, dtype=grad_dtype, device=device)
+        Gt = None if step_grad_dtype == grad_dtype else \
+            torch.zeros(layout.seg, dtype=step_grad_dtype, device=device)
+        return cls(W, M, Gf, Gs, Gt)
+
+
+def sharded_step_bucketed(layout: BucketedLayout, bufs: Sequence[BucketBuffers], rank: int,
+                          step_fns: Sequence[Callable], group=None, comm_stream=None,
+                          to_step_dtype: Optional[Callable] = None):
+    """One data-parallel Muon step over the buckets of `layout`.
+
+      1. the reduce-scatters of every bucket's gradients are issued at once, in
+         bucket order, on `comm_stream` (after the gradients on the current
+         stream are ready);
+      2. for each bucket in order, the current stream waits for that bucket's
+         reduce-scatter only, rounds the summed gradients to the step's dtype
+         with `to_step_dtype(G_step, G_seg)` if the reduction ran in another
+         dtype, and runs `step_fns[b](W_views, M_views, G_views)` on views of
+         this rank's segment; so bucket b's step overlaps the reduce-scatters
+         of the buckets after it;
+      3. the all-gathers of the updated weights are issued on `comm_stream` in
+         bucket order, each waiting for its own bucket's step only, so that
+         bucket b's all-gather overlaps the steps of the buckets after it;
+         the current stream finally waits for all of them.
+
+    Every rank issues the same collectives in the same order (all
+    reduce-scatters, then all all-gathers).  On CPU tensors (gloo) the waits
+    are host waits and `comm_stream` must be None."""
+    import torch
+    import torch.distributed as dist
+    cuda = bufs[0].W_flat.is_cuda
+    if comm_stream is not None and not cuda:
+        raise ValueError("comm_stream needs CUDA buffers")
+    compute = torch.cuda.current_stream() if cuda else None
+    side = torch.cuda.stream(comm_stream) if comm_stream is not None else nullcontext()
+    if comm_stream is not None:
+        comm_stream.wait_stream(compute)
+    with side:
+        rs = [dist.reduce_scatter_tensor(bf.G_seg, bf.G_flat, op=dist.ReduceOp.SUM,
+                                         group=group, async_op=True) for bf in bufs]
+    done = []
+    for b, (L, bf) in enumerate(zip(layout.layouts, bufs)):
+        rs[b].wait()
+        if bf.G_step is not bf.G_seg:
+            if to_step_dtype is None:
+                raise ValueError("a reduction dtype other than the step's needs "
+                                 "to_step_dtype")
+            to_step_dtype(bf.G_step, bf.G_seg)
+        own = bf.W_flat[rank * L.seg:(rank + 1) * L.seg]
+        if L.mine[rank]:
+            step_fns[b](L.local_views(own, rank), L.local_views(bf.M_seg, rank),
+                        L.local_views(bf.G_step, rank))
+        if comm_stream is not None:
+            ev = torch.cuda.Event()
+            ev.record(compute)
+            done.append(ev)
+    ag = []
+    with side:
+        for b, (L, bf) in enumerate(zip(layout.layouts, bufs)):
+            if comm_stream is not None:
+                comm_stream.wait_event(done[b])
+            own = bf.W_flat[rank * L.seg:(rank + 1) * L.seg]
+            ag.append(dist.all_gather_into_tensor(bf.W_flat, own.clone(), group=group,
+                                                  async_op=True))
+    for w in ag:
+        w.wait()
 
 
 def max_over_ranks(value: float, device=None, group=None) -> float:

@@ -1,6 +1,7 @@
 // Host-side check of the Newton-Schulz list scheduler (schedule.h): reads
-// "n_mats steps clusters" then n_mats lines "rows cols" on stdin, builds the
-// schedule and prints one line per item "mat mode k ti tj kt", then
+// "n_mats steps clusters group_bytes lag" (group_bytes < 0: the library's
+// default order) then n_mats lines "rows cols" on stdin, builds the schedule
+// and prints one line per item "mat mode k ti tj kt", then
 // "makespan <simulated cycles>".
 #include <cstdio>
 #include <vector>
@@ -10,8 +11,11 @@
 using namespace muonb200;
 
 int main() {
-  int n_mats = 0, steps = 0, clusters = 0;
-  if (std::scanf("%d %d %d", &n_mats, &steps, &clusters) != 3) return 2;
+  int n_mats = 0, steps = 0, clusters = 0, lag = 0;
+  double group_bytes = 0.0;
+  if (std::scanf("%d %d %d %lf %d", &n_mats, &steps, &clusters, &group_bytes, &lag) != 5)
+    return 2;
+  const SchedPolicy pol = group_bytes < 0 ? default_policy() : SchedPolicy{group_bytes, lag};
   std::vector<SchedMatrix> mats(n_mats);
   long long per_step = 0;
   for (int i = 0; i < n_mats; ++i) {
@@ -26,9 +30,9 @@ int main() {
   }
   std::vector<SchedItem> out(per_step * steps);
   std::vector<SchedGroup> groups(static_cast<size_t>(n_mats) * steps * 3);
-  std::vector<int> order(n_mats);
+  std::vector<int> order(2 * static_cast<size_t>(n_mats) + 1);
   std::vector<double> cl(clusters);
-  const long long n = build_schedule(mats.data(), n_mats, steps, clusters, out.data(),
+  const long long n = build_schedule(mats.data(), n_mats, steps, clusters, pol, out.data(),
                                      static_cast<long long>(out.size()), groups.data(),
                                      order.data(), cl.data());
   if (n < 0) return 3;

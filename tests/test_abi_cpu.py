@@ -58,7 +58,11 @@ def test_library_has_no_driver_or_torch_dependency():
 
 
 def test_constants(L):
-    assert L.muon_abi_version() == 100
+    assert L.muon_abi_version() == 101
+    import torch
+    if not torch.cuda.is_available():
+        # no plan can be created without a device, so nothing was allocated
+        assert L.muon_device_allocation_count() == 0
     assert binding.status_string(0) == "ok"
     assert "timed out" in binding.status_string(-5)
     assert binding.status_string(-99) == "unknown status"

@@ -113,6 +113,22 @@ def test_heavy_tailed_rows():
         check_step(g, step, [0, 1], emu_tol=1e-2)
 
 
+def test_later_plan_needing_less_staging_leaves_earlier_plan_working():
+    """The prologue kernels' dynamic shared memory limit is a per-device
+    setting of each kernel, shared by every plan.  A plan created later whose
+    transposed items need less staging (here about 1 KB against 33 KB and
+    19 KB) must not lower it below what an earlier plan launches with: the
+    earlier plan's steps still run and match the oracle."""
+    big = wl.custom([(2048, 512), (700, 300)], H, Q5, grad_std=1.0, wid=520)
+    g_big = GpuMuon(big)          # one-pass and two-pass transposed items
+    small = wl.custom([(64, 16), (40, 12)], H, Q5, grad_std=1.0, wid=521)
+    g_small = GpuMuon(small)
+    check_step(g_small, 0, [0, 1])
+    check_step(g_big, 0, [0, 1])
+    check_step(g_small, 1, [0, 1])
+    check_step(g_big, 1, [0, 1])
+
+
 def test_deterministic():
     import torch
     outs = []

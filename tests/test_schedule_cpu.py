@@ -10,6 +10,7 @@ from collections import Counter, defaultdict
 
 import pytest
 
+import tables
 from muon_optimizer_step_02_b200 import workloads as wl
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -29,8 +30,9 @@ def exe(tmp_path_factory):
     return out
 
 
-def run(exe, shapes, steps, clusters):
-    inp = f"{len(shapes)} {steps} {clusters}\n" + "".join(
+def run(exe, shapes, steps, clusters, group_bytes=-1.0, lag=0):
+    """The list for a policy (group_bytes < 0: the library's default)."""
+    inp = f"{len(shapes)} {steps} {clusters} {group_bytes} {lag}\n" + "".join(
         f"{r} {c}\n" for r, c in shapes)
     res = subprocess.run([exe], input=inp, capture_output=True, text=True,
                          check=True)
@@ -117,10 +119,29 @@ def phase_major_makespan(shapes, steps, clusters):
                                                  (4, 5, 74), (1, 5, 74),
                                                  (5, 5, 74)])
 def test_schedule_valid_and_no_worse(exe, widx, steps, clusters):
-    shapes = wl.workload(widx).shapes
+    shapes = tables.workload(widx).shapes
     items, makespan = run(exe, shapes, steps, clusters)
     check(items, shapes, steps)
     assert makespan <= phase_major_makespan(shapes, steps, clusters) * 1.001
+
+
+@pytest.mark.parametrize("group_mb,lag", [(15, 1), (15, 3), (31, 6), (0.001, 1)])
+def test_wave_orders_are_valid(exe, group_mb, lag):
+    """The wave orders (groups of consecutive matrices started `lag` phase
+    slots apart) keep every dependency before its readers too."""
+    for widx in (2, 4):
+        shapes = tables.workload(widx).shapes
+        items, _ = run(exe, shapes, 5, 74, group_mb * 2 ** 20, lag)
+        check(items, shapes, 5)
+    shapes = [(1, 1), (7, 13), (300, 200), (129, 257), (1000, 8), (513, 1025)]
+    for steps, clusters in ((1, 1), (3, 2), (5, 7)):
+        items, _ = run(exe, shapes, steps, clusters, group_mb * 2 ** 20, lag)
+        check(items, shapes, steps)
+
+
+def test_default_order_is_phase_major(exe):
+    shapes = tables.workload(2).shapes
+    assert run(exe, shapes, 5, 74) == run(exe, shapes, 5, 74, 1e30, 0)
 
 
 def test_schedule_ragged_and_few_clusters(exe):

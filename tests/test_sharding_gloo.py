@@ -1,7 +1,8 @@
-"""Multi-process host logic on CPU (gloo, world size 2): matrix ownership,
-the reduce / step / broadcast exchange of a sharded step, and the benchmark's
-max-over-ranks timing.  The per-rank compute is the fp64 oracle here; on GPUs
-it is the library's step."""
+"""Multi-process host logic on CPU (gloo, world sizes 2 and 4): matrix
+ownership, the flat reduce-scatter / owner step / all-gather exchange of a
+sharded step, its bucketed form (with the gradient reduction in fp32 as an
+option), and the benchmark's max-over-ranks timing.  The per-rank compute is
+the fp64 oracle here; on GPUs it is the library's step."""
 import os
 import socket
 
@@ -34,77 +35,6 @@ def _free_port():
     port = s.getsockname()[1]
     s.close()
     return port
-
-
-def _worker(rank, world, port, q):
-    import oracle.muon_oracle as mo
-    os.environ["MASTER_ADDR"] = "127.0.0.1"
-    os.environ["MASTER_PORT"] = str(port)
-    dist.init_process_group("gloo", rank=rank, world_size=world,
-                            init_method=f"tcp://127.0.0.1:{port}")
-    try:
-        shapes = [(48, 32), (32, 48), (40, 40), (16, 64), (64, 16), (24, 24)]
-        h = wl.Hyper(momentum=0.9, lr=0.05, weight_decay=0.1)
-        coeffs = [wl.FIXED_QUINTIC] * 3
-        w = wl.custom(shapes, h, coeffs, grad_std=1.0, wid=400)
-        owner = sharding.partition_matrices(shapes, world, 3)
-        W = [torch.from_numpy(wl.weight(w, i).astype(np.float64))
-             for i in range(len(shapes))]
-        M = [torch.zeros_like(x) for x in W]
-        hyp = mo.MuonHyper(momentum=h.momentum, lr=h.lr,
-                           weight_decay=h.weight_decay)
-        for step in range(2):
-            # rank r holds a share of the gradient: the shares sum to G
-            G = [wl.bf16_bits_to_f32(wl.grad_bits(w, i, step)).astype(np.float64)
-                 for i in range(len(shapes))]
-            G_local = [torch.from_numpy(g * (0.25 if rank == 0 else 0.75))
-                       for g in G]
-
-            def step_fn(idx):
-                for i in idx:
-                    Wn, Mn, _ = mo.muon_step(W[i].numpy(), M[i].numpy(),
-                                             G_local[i].numpy(), hyp, coeffs,
-                                             1.0)
-                    W[i].copy_(torch.from_numpy(Wn))
-                    M[i].copy_(torch.from_numpy(Mn))
-
-            sharding.sharded_step(W, M, G_local, owner, rank, step_fn)
-        t = sharding.max_over_ranks(1.0 + rank)
-        q.put((rank, [x.numpy().copy() for x in W], t))
-    finally:
-        dist.destroy_process_group()
-
-
-def test_sharded_step_matches_single_process():
-    import oracle.muon_oracle as mo
-    world = 2
-    port = _free_port()
-    ctx = mp.get_context("spawn")
-    q = ctx.Queue()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, q))
-             for r in range(world)]
-    for p in procs:
-        p.start()
-    out = [q.get(timeout=120) for _ in range(world)]
-    for p in procs:
-        p.join(timeout=60)
-        assert p.exitcode == 0
-    # single-process reference
-    shapes = [(48, 32), (32, 48), (40, 40), (16, 64), (64, 16), (24, 24)]
-    h = wl.Hyper(momentum=0.9, lr=0.05, weight_decay=0.1)
-    coeffs = [wl.FIXED_QUINTIC] * 3
-    w = wl.custom(shapes, h, coeffs, grad_std=1.0, wid=400)
-    hyp = mo.MuonHyper(momentum=h.momentum, lr=h.lr, weight_decay=h.weight_decay)
-    W = [wl.weight(w, i).astype(np.float64) for i in range(len(shapes))]
-    M = [np.zeros_like(x) for x in W]
-    for step in range(2):
-        for i in range(len(shapes)):
-            G = wl.bf16_bits_to_f32(wl.grad_bits(w, i, step)).astype(np.float64)
-            W[i], M[i], _ = mo.muon_step(W[i], M[i], G, hyp, coeffs, 1.0)
-    for rank, Ws, t in out:
-        assert t == 2.0            # max over ranks of 1.0 + rank
-        for a, b in zip(Ws, W):
-            np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
 
 
 def test_flat_layout_is_owner_ordered_and_aligned():
@@ -159,7 +89,8 @@ def _flat_worker(rank, world, port, q):
                 g = wl.bf16_bits_to_f32(wl.grad_bits(w, i, step)).astype(np.float64)
                 v.copy_(torch.from_numpy(g * share))
             sharding.sharded_step_flat(L, W_flat, M_seg, G_flat, G_seg, rank, step_fn)
-        q.put((rank, [v.numpy().copy() for v in L.views(W_flat)]))
+        t = sharding.max_over_ranks(1.0 + rank)
+        q.put((rank, [v.numpy().copy() for v in L.views(W_flat)], t))
     finally:
         dist.destroy_process_group()
 
@@ -189,6 +120,102 @@ def test_flat_sharded_step_matches_single_process(world):
         for i in range(len(shapes)):
             G = wl.bf16_bits_to_f32(wl.grad_bits(w, i, step)).astype(np.float64)
             W[i], M[i], _ = mo.muon_step(W[i], M[i], G, hyp, coeffs, 1.0)
+    for rank, Ws, t in out:
+        assert t == float(world)           # max over ranks of 1.0 + rank
+        for a, b in zip(Ws, W):
+            np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
+
+
+SHAPES_B = [(48, 32), (32, 48), (40, 40), (16, 64), (64, 16), (24, 24), (8, 100),
+            (56, 24), (24, 56)]
+
+
+def _bucket_worker(rank, world, port, q, n_buckets, fp32_reduce):
+    import oracle.muon_oracle as mo
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            init_method=f"tcp://127.0.0.1:{port}")
+    try:
+        h = wl.Hyper(momentum=0.9, lr=0.05, weight_decay=0.1)
+        coeffs = [wl.FIXED_QUINTIC] * 3
+        w = wl.custom(SHAPES_B, h, coeffs, grad_std=1.0, wid=402)
+        BL = sharding.BucketedLayout(SHAPES_B, world, n_buckets, 3)
+        gdt = torch.float32 if fp32_reduce else torch.float64
+        bufs = [sharding.BucketBuffers.allocate(L, torch.float64, gdt, torch.float64)
+                for L in BL.layouts]
+        for bk, L, bf in zip(BL.buckets, BL.layouts, bufs):
+            for j, v in enumerate(L.views(bf.W_flat)):
+                v.copy_(torch.from_numpy(wl.weight(w, bk[j]).astype(np.float64)))
+        hyp = mo.MuonHyper(momentum=h.momentum, lr=h.lr, weight_decay=h.weight_decay)
+
+        def step_fn(Wv, Mv, Gv):
+            for a, m, g in zip(Wv, Mv, Gv):
+                Wn, Mn, _ = mo.muon_step(a.numpy(), m.numpy(), g.numpy(), hyp, coeffs, 1.0)
+                a.copy_(torch.from_numpy(Wn))
+                m.copy_(torch.from_numpy(Mn))
+
+        def to_bf16_values(dst, src):
+            # the library rounds the fp32 sum to bf16; the fp64 step reads it
+            dst.copy_(src.to(torch.bfloat16).to(torch.float64))
+
+        share = SHARES[world][rank]
+        for step in range(2):
+            for bk, L, bf in zip(BL.buckets, BL.layouts, bufs):
+                bf.G_flat.zero_()
+                for j, v in enumerate(L.views(bf.G_flat)):
+                    g = wl.bf16_bits_to_f32(wl.grad_bits(w, bk[j], step)).astype(np.float64)
+                    v.copy_(torch.from_numpy(g * share))
+            sharding.sharded_step_bucketed(BL, bufs, rank, [step_fn] * n_buckets,
+                                           to_step_dtype=to_bf16_values if fp32_reduce
+                                           else None)
+        W = [None] * len(SHAPES_B)
+        for bk, L, bf in zip(BL.buckets, BL.layouts, bufs):
+            for j, v in enumerate(L.views(bf.W_flat)):
+                W[bk[j]] = v.numpy().copy()
+        q.put((rank, W))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bucketed_layout_covers_every_matrix_once():
+    shapes = wl.workload(2).shapes
+    for world in (1, 2, 8):
+        for nb in (1, 2, 3, 11, 66):
+            BL = sharding.BucketedLayout(shapes, world, nb)
+            assert len(BL.buckets) == nb
+            flat = [i for bk in BL.buckets for i in bk]
+            assert flat == list(range(len(shapes)))      # consecutive, in order
+            assert all(bk for bk in BL.buckets)
+    with pytest.raises(ValueError):
+        sharding.BucketedLayout(shapes, 2, 0)
+
+
+@pytest.mark.parametrize("world,n_buckets,fp32_reduce",
+                         [(2, 2, False), (2, 3, True), (4, 3, False), (4, 2, True)])
+def test_bucketed_sharded_step_matches_single_process(world, n_buckets, fp32_reduce):
+    import oracle.muon_oracle as mo
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_bucket_worker,
+                         args=(r, world, port, q, n_buckets, fp32_reduce))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    h = wl.Hyper(momentum=0.9, lr=0.05, weight_decay=0.1)
+    coeffs = [wl.FIXED_QUINTIC] * 3
+    w = wl.custom(SHAPES_B, h, coeffs, grad_std=1.0, wid=402)
+    hyp = mo.MuonHyper(momentum=h.momentum, lr=h.lr, weight_decay=h.weight_decay)
+    W = [wl.weight(w, i).astype(np.float64) for i in range(len(SHAPES_B))]
+    M = [np.zeros_like(x) for x in W]
+    for step in range(2):
+        for i in range(len(SHAPES_B)):
+            G = wl.bf16_bits_to_f32(wl.grad_bits(w, i, step)).astype(np.float64)
+            W[i], M[i], _ = mo.muon_step(W[i], M[i], G, hyp, coeffs, 1.0)
     for rank, Ws in out:
         for a, b in zip(Ws, W):
+            # dyadic shares of bf16 values sum exactly in fp32 and in fp64
             np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
