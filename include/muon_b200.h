@@ -65,7 +65,8 @@ typedef enum {
   MUON_ERR_ALIGNMENT = -3,   /* a device pointer is not 16-byte aligned      */
   MUON_ERR_CUDA = -4,        /* CUDA runtime/driver error (launch, encode)   */
   MUON_ERR_TIMEOUT = -5,     /* a device-side bounded wait ran out           */
-  MUON_ERR_WORKSPACE = -6    /* workspace null, too small or misaligned      */
+  MUON_ERR_WORKSPACE = -6,   /* workspace null, too small or misaligned      */
+  MUON_ERR_DEVICE_CHECK = -7 /* device-checked build: an index out of bounds */
 } muon_status_t;
 
 /* Opaque plan: matrix shapes, schedule tables and a small device table. */
@@ -237,7 +238,8 @@ muon_status_t muon_f32_to_bf16(uint16_t *dst, const float *src, int64_t n,
 
 /* Synchronises `stream`, reads and clears the plan's device error word.
  * Returns MUON_ERR_TIMEOUT if a kernel gave up on a bounded wait since the
- * last call, MUON_ERR_CUDA on a CUDA error, MUON_OK otherwise. */
+ * last call, MUON_ERR_DEVICE_CHECK if a device check of the checked build
+ * failed, MUON_ERR_CUDA on a CUDA error, MUON_OK otherwise. */
 muon_status_t muon_get_last_error(muon_plan_t *plan, muon_stream_t stream);
 
 /* Enqueues on `stream` a copy of the plan's device error word into
@@ -288,13 +290,25 @@ int32_t ema_update_launches(int32_t n_tensors);
  * advanced). */
 int32_t adamw_ema_launches(int32_t n_tensors, int32_t with_step_dev);
 
+/* 1 if this library is the device-checked build (compiled with
+ * MUON_DEVICE_CHECKS): every work item the kernels decode is checked
+ * against its matrix's tile grid and every epilogue store against its
+ * buffer before the access; a failure skips the access, records the error
+ * word and the offending index, stops the tensor-core kernel like a failed
+ * wait, and muon_get_last_error returns MUON_ERR_DEVICE_CHECK.  0 for the
+ * default build, which carries none of these checks. */
+int32_t muon_device_checks(void);
+
 /* Test hooks.  Fault 1 makes the tensor-core kernel's load warp skip one
  * stage of its first tile in block 0, so that the consumer's bounded wait
  * runs out and the timeout path is exercised (MUON_ERR_TIMEOUT from
  * muon_get_last_error).  Fault 2 asks for more dynamic shared memory than the
  * tensor-core kernel was set up for, so that the runtime refuses its launch
  * and the step call returns MUON_ERR_CUDA (no kernel of it runs; the earlier
- * launches of the call do).  0 turns them off. */
+ * launches of the call do).  Fault 3, accepted only by the device-checked
+ * build (MUON_ERR_UNSUPPORTED otherwise), uploads the work list with its
+ * last item moved outside its matrix, which the kernel's checks must catch.
+ * 0 turns them off. */
 muon_status_t muon_plan_set_fault(muon_plan_t *plan, int32_t fault);
 
 /* ABI version (major * 100 + minor). */

@@ -20,6 +20,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmuonb200.so")
+# The same sources with MUON_DEVICE_CHECKS: every work item and epilogue
+# store checked on the device before the access (tests and debugging).
+LIB_CHECKED = os.path.join(PKG, "libmuonb200_checked.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -35,10 +38,10 @@ def sources():
                   glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def is_stale() -> bool:
-    if not os.path.exists(LIB):
+def is_stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(s) > t for s in sources())
 
 
@@ -49,18 +52,28 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found: cannot build libmuonb200.so")
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not is_stale():
-        return LIB
+def _compile(lib: str, extra, verbose: bool):
     cu = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
-    tmp = LIB + ".tmp"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *cu]
+    tmp = lib + ".tmp"
+    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *cu]
     if verbose:
         print(" ".join(cmd), flush=True)
-    res = subprocess.run(cmd, capture_output=True, text=True)
-    if res.returncode != 0:
-        raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
-    os.replace(tmp, LIB)
+    return tmp, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.PIPE,
+                                 text=True)
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Builds the default library and the device-checked one (in parallel)
+    when their sources changed; returns the default library's path."""
+    jobs = []
+    for lib, extra in ((LIB, []), (LIB_CHECKED, ["-DMUON_DEVICE_CHECKS"])):
+        if force or is_stale(lib):
+            jobs.append((lib, *_compile(lib, extra, verbose)))
+    for lib, tmp, proc in jobs:
+        out, err = proc.communicate()
+        if proc.returncode != 0:
+            raise RuntimeError("nvcc failed:\n" + out + err)
+        os.replace(tmp, lib)
     return LIB
 
 

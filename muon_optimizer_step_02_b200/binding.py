@@ -13,8 +13,11 @@ from ctypes import (POINTER, Structure, c_char_p, c_double, c_float, c_int32,
                     c_int64, c_size_t, c_void_p)
 from typing import List, Optional, Sequence, Tuple
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
-                        "libmuonb200.so")
+_PKG = os.path.dirname(os.path.abspath(__file__))
+# MUONB200_LIB selects another build of the library, e.g. the device-checked
+# one (CHECKED_LIB_PATH), for a whole process.
+LIB_PATH = os.environ.get("MUONB200_LIB") or os.path.join(_PKG, "libmuonb200.so")
+CHECKED_LIB_PATH = os.path.join(_PKG, "libmuonb200_checked.so")
 
 MUON_OK = 0
 MUON_ERR_INVALID_ARG = -1
@@ -23,6 +26,7 @@ MUON_ERR_ALIGNMENT = -3
 MUON_ERR_CUDA = -4
 MUON_ERR_TIMEOUT = -5
 MUON_ERR_WORKSPACE = -6
+MUON_ERR_DEVICE_CHECK = -7
 
 KIND_NAMES = ("prologue", "gram", "poly", "apply", "final", "ns", "scale")
 
@@ -145,6 +149,8 @@ def lib():
     L.muon_noalloc_set_fault.restype = c_int32
     L.muon_f32_to_bf16.argtypes = [c_void_p, c_void_p, c_int64, c_void_p]
     L.muon_f32_to_bf16.restype = c_int32
+    L.muon_device_checks.argtypes = []
+    L.muon_device_checks.restype = c_int32
     L.muon_device_allocation_count.argtypes = []
     L.muon_device_allocation_count.restype = c_int64
     _lib = L

@@ -10,8 +10,20 @@
 namespace muonb200 {
 
 constexpr int kEpiWarps = 8;                 // two per TMEM lane quadrant
-// producer warp, MMA warp, epilogue warps, completion-signal warp
-constexpr int kNsThreads = 96 + 32 * kEpiWarps;
+// Warpgroup 0: producer warp, MMA warp, completion-signal warp, one idle
+// warp; warpgroups 1 and 2: the epilogue warps.
+constexpr int kEpiWarp0 = 4;                 // first epilogue warp
+constexpr int kNsThreads = 32 * (kEpiWarp0 + kEpiWarps);
+// Register split after set-up (setmaxnreg): the launch gives every thread
+// kNsRegsLaunch registers (384 threads x 168 = 64,512 of the SM's 65,536);
+// warpgroup 0 returns all but kNsRegsControl and the two epilogue
+// warpgroups take them, 128 x 56 + 256 x 224 = 64,512: the sum never
+// exceeds what the block was launched with, so the increase cannot wait.
+constexpr int kNsRegsLaunch = 168;
+constexpr int kNsRegsControl = 56;
+constexpr int kNsRegsEpilogue = 224;
+static_assert(128 * kNsRegsControl + 256 * kNsRegsEpilogue <= kNsThreads * kNsRegsLaunch,
+              "register split exceeds the launch allocation");
 
 
 

@@ -25,12 +25,14 @@
 // s = 1 / (||X~||_F + eps_frob) in step 0 (the Frobenius normalisation folded
 // into the first products), 1 afterwards.
 //
-// Roles (320 threads per CTA): warp 0 issues TMA loads (.cta_group::2, no
-// multicast) into a 6-stage ring, counting both CTAs' bytes on the leader's
-// barrier; warp 1 of the leader issues the pair MMAs from one thread and
-// frees stages / hands over accumulators with multicast tcgen05.commit;
-// warps 2-9 of each CTA drain that CTA's 128 TMEM lanes and run the fused
-// epilogue.  All waits are bounded: a failure raises both CTAs' abort flags
+// Roles (384 threads per CTA, three warpgroups): warp 0 issues TMA loads
+// (.cta_group::2, no multicast) into a 6-stage ring, counting both CTAs'
+// bytes on the leader's barrier; warp 1 of the leader issues the pair MMAs
+// from one thread and frees stages / hands over accumulators with multicast
+// tcgen05.commit; warp 2 publishes completed items; warp 3 idles; warps 4-11
+// (warpgroups 1 and 2) drain that CTA's 128 TMEM lanes and run the fused
+// epilogue.  After set-up warpgroup 0 gives its registers to the epilogue
+// warpgroups (setmaxnreg), which then hold their blocks without spilling.  All waits are bounded: a failure raises both CTAs' abort flags
 // and the global error word, and every CTA still meets the final cluster
 // barrier before TMEM is freed.
 //
@@ -44,6 +46,7 @@
 
 #include "k_ns_common.cuh"
 #include "muon_types.cuh"
+#include "schedule.h"
 #include "sm100_ptx.cuh"
 
 namespace muonb200 {
@@ -54,10 +57,12 @@ constexpr int kMegaStages = 6;
 struct MegaParams {
   const MatDev* mats;
   const SchedItem* items; // the schedule (host-built list, see schedule.h)
-  const float* mat_scale; // per-matrix Frobenius scale from the prologue
-  int32_t* err;
+  const float* partials;  // the prologue's Frobenius partial sums
+  int32_t* step_inc;      // scheduled step counter to advance, or null
+  int32_t* err;           // error word, then the index of a failed check
   int32_t* done;          // [mat][step][phase] completion counts, zeroed
   int32_t n_items;
+  int32_t n_mats;
   int32_t steps;
   int32_t fault, fresh;
   float a[kMegaMaxSteps], b[kMegaMaxSteps], c[kMegaMaxSteps];
@@ -103,21 +108,43 @@ __device__ __forceinline__ bool wait_count(const int32_t* ctr, int32_t target,
   }
 }
 
+// s = 1 / (||X~||_F + eps) of a matrix from its prologue partials: lane l
+// adds slots l, l + 32, ..., then the warp's butterfly adds the lanes -- a
+// fixed order, the same in every warp and on every run.
+__device__ __forceinline__ float frob_scale(const float* partials, const MatDev* md,
+                                            int lane, float eps) {
+  float s = 0.f;
+  for (int i = lane; i < md->part_count; i += 32) s += partials[md->part_first + i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return 1.f / (sqrtf(s) + eps);
+}
+
 struct MegaItem {
   NsTile tl;
   int mode;
   int k;
+  int dep_target;   // completion count of the phase it reads (0: none)
 };
 
-__device__ __forceinline__ MegaItem mega_item(const MegaParams& p, int g) {
-  const SchedItem si = p.items[g];
+// The raw 16-byte record of list position g (zeros past the end), read with
+// one vector load.  Each role loads the record of its next item while it
+// works on the current one, so no item starts with a global-memory round
+// trip for its own description.
+__device__ __forceinline__ uint4 load_item_raw(const MegaParams& p, int g) {
+  if (g >= p.n_items) return make_uint4(0u, 0u, 0u, 0u);
+  return __ldg(reinterpret_cast<const uint4*>(p.items) + g);
+}
+
+__device__ __forceinline__ MegaItem unpack_item(const uint4 r) {
   MegaItem it;
-  it.tl.mat = si.mat;
-  it.tl.ti = si.ti;
-  it.tl.tj = si.tj;
-  it.tl.kt = si.kt;
-  it.mode = si.mode;
-  it.k = si.k;
+  it.tl.mat = static_cast<uint16_t>(r.x & 0xFFFFu);
+  it.tl.ti = static_cast<uint16_t>(r.x >> 16);
+  it.tl.tj = static_cast<uint16_t>(r.y & 0xFFFFu);
+  it.tl.kt = static_cast<uint16_t>(r.y >> 16);
+  it.mode = static_cast<int>(r.z & 0xFFu);
+  it.k = static_cast<int>((r.z >> 8) & 0xFFu);
+  it.dep_target = static_cast<int>(r.w);
   return it;
 }
 
@@ -126,18 +153,13 @@ __device__ __forceinline__ int32_t* done_counter(const MegaParams& p, int mat,
   return p.done + (static_cast<size_t>(mat) * p.steps + k) * 3 + mode;
 }
 
-// Completion count an item must see before it reads its inputs; nullptr if
-// it has no in-kernel dependency (gram of step 0 reads the prologue's X).
+// The completion counter of the phase an item reads (it.dep_target counts
+// its tiles); nullptr if it has no in-kernel dependency (the gram of step 0
+// reads the prologue's X).
 __device__ __forceinline__ const int32_t* dep_counter(const MegaParams& p,
-                                                      const MegaItem& it,
-                                                      const MatDev* md,
-                                                      int32_t& target) {
-  if (it.mode == kModeGram) {
-    if (it.k == 0) return nullptr;
-    target = 2 * md->n_apply_tiles;
-    return done_counter(p, it.tl.mat, it.k - 1, kModeApply);
-  }
-  target = 2 * md->n_sym_tiles;
+                                                      const MegaItem& it) {
+  if (it.dep_target == 0) return nullptr;
+  if (it.mode == kModeGram) return done_counter(p, it.tl.mat, it.k - 1, kModeApply);
   return done_counter(p, it.tl.mat, it.k, it.mode == kModePoly ? kModeGram : kModePoly);
 }
 
@@ -188,10 +210,23 @@ __device__ __forceinline__ void load_w_block(const MatDev* md, int row0, int col
 // W <- W decay - step O on the block of load_w_block: wv holds its W, v the
 // accumulator row of this lane (O); O also goes to the optional update
 // output.  `stage` is the warp's 32 x 32 fp32 shared staging block.
+// Device-checked build: a weight store outside the rows x cols matrix is
+// skipped and its offset recorded.
+__device__ __forceinline__ bool w_store_ok(const MatDev* md, size_t off, int width,
+                                           int32_t* err) {
+  if constexpr (!kDeviceChecks) {
+    return true;
+  } else {
+    if (off + width <= static_cast<size_t>(md->rows) * md->cols) return true;
+    record_check_failure(err, kErrCheckStore, static_cast<int32_t>(off));
+    return false;
+  }
+}
+
 __device__ __forceinline__ void store_w_block(const MatDev* md, int row0, int col0,
                                               int lane, float decay, float step,
                                               const float (&wv)[32], const float (&v)[32],
-                                              float* stage) {
+                                              float* stage, int32_t* err) {
   const int m = md->m, n = md->n;
   float* __restrict__ w = md->w;
   float* __restrict__ out = md->out;
@@ -211,6 +246,7 @@ __device__ __forceinline__ void store_w_block(const MatDev* md, int row0, int co
       const int rr = 4 * i + (lane >> 3);
       const float4 o4 = *reinterpret_cast<const float4*>(stage + rr * 32 + 4 * (c ^ (rr & 7)));
       const size_t g = g0 + static_cast<size_t>(4 * i) * n;
+      if (!w_store_ok(md, g, 4, err)) continue;
       *reinterpret_cast<float4*>(w + g) =
           make_float4(fmaf(wv[4 * i], decay, -step * o4.x),
                       fmaf(wv[4 * i + 1], decay, -step * o4.y),
@@ -227,7 +263,7 @@ __device__ __forceinline__ void store_w_block(const MatDev* md, int row0, int co
     const size_t g = static_cast<size_t>(row) * n + col0;
 #pragma unroll
     for (int e = 0; e < 32; ++e)
-      if (col0 + e < n) {
+      if (col0 + e < n && w_store_ok(md, g + e, 1, err)) {
         w[g + e] = fmaf(wv[e], decay, -step * v[e]);
         if (out) out[g + e] = v[e];
       }
@@ -236,6 +272,7 @@ __device__ __forceinline__ void store_w_block(const MatDev* md, int row0, int co
     for (int e = 0; e < 32; ++e)
       if (col0 + e < n) {
         const size_t off = static_cast<size_t>(col0 + e) * m + row;
+        if (!w_store_ok(md, off, 1, err)) continue;
         w[off] = fmaf(wv[e], decay, -step * v[e]);
         if (out) out[off] = v[e];
       }
@@ -301,6 +338,16 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // The kernel is launched as a programmatic dependent of the prologue: the
+  // set-up above overlaps the prologue's last blocks; everything below reads
+  // what the prologue wrote (X~, the Frobenius partials, the zeroed
+  // counters, the scheduled learning rate), so every thread waits for it to
+  // complete here.  The EMA launched after this kernel may then get its
+  // blocks resident; they wait in turn for this grid to finish.
+  grid_dependency_wait();
+  grid_launch_dependents();
+  // The prologue has read the scheduled step number; advance it once.
+  if (p.step_inc != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.step_inc += 1;
   const uint32_t peer_abort = mapa_shared(smem_addr(const_cast<int*>(abort_flag)), rank ^ 1u);
   const uint32_t leader_full0 = mapa_shared(full_bar(0), 0);
   auto fail = [&](int32_t code) {
@@ -308,14 +355,46 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
     *abort_flag = 1;
     st_shared_cluster_u32(peer_abort, 1u);
   };
+  // Device-checked build: an item outside its matrix's tile grid (or with
+  // the wrong K extent or dependency target) is never touched; its list
+  // position is recorded and the kernel aborts like a failed wait.
+  auto item_ok = [&](const MegaItem& it, int g) -> bool {
+    if constexpr (!kDeviceChecks) {
+      return true;
+    } else {
+      bool valid = it.tl.mat < p.n_mats;
+      if (valid) {
+        const MatDev* md = p.mats + it.tl.mat;
+        valid = sched_item_valid(it.mode, it.k, it.tl.ti, it.tl.tj, it.tl.kt,
+                                 it.dep_target, md->m, md->n, p.steps);
+      }
+      if (!valid) {
+        record_check_failure(p.err, kErrCheckItem, g);
+        *abort_flag = 1;
+        st_shared_cluster_u32(peer_abort, 1u);
+      }
+      return valid;
+    }
+  };
 
+  if (warp < kEpiWarp0) {
+  // Warpgroup 0 keeps few registers; the epilogue warpgroups take the rest.
+  // (The change sits at the top of each warpgroup's branch, so that the
+  // compiler gives each branch its own register budget.)
+  regs_decrease<kNsRegsControl>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int it = 0;
       bool ok = true;
+      uint4 nx = load_item_raw(p, pair);
       for (int g = pair; ok && g < total; g += npairs) {
-        const MegaItem item = mega_item(p, g);
+        const MegaItem item = unpack_item(nx);
+        nx = load_item_raw(p, g + npairs);
+        if (!item_ok(item, g)) {
+          ok = false;
+          break;
+        }
         const NsTile tl = item.tl;
         const MatDev* md = p.mats + tl.mat;
         const int src = item.k & 1;
@@ -335,10 +414,9 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
           tensormap_acquire(tm_a);
           if (tm_b != tm_a) tensormap_acquire(tm_b);
         }
-        int32_t target = 0;
-        const int32_t* dep = dep_counter(p, item, md, target);
+        const int32_t* dep = dep_counter(p, item);
         if (dep != nullptr) {
-          if (!wait_count(dep, target, abort_flag, p.err)) {
+          if (!wait_count(dep, item.dep_target, abort_flag, p.err)) {
             fail(kErrTimeoutProducer);
             ok = false;
             break;
@@ -390,8 +468,11 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
       constexpr uint32_t idesc_mn = idesc_bf16_f32_pair(kPairTile, true);
       int it = 0, lt = 0;
       bool ok = true;
+      uint4 nx = load_item_raw(p, pair);
       for (int g = pair; ok && g < total; g += npairs, ++lt) {
-        const MegaItem item = mega_item(p, g);
+        const MegaItem item = unpack_item(nx);
+        nx = load_item_raw(p, g + npairs);
+        if (!item_ok(item, g)) break;
         const bool bmn = item.mode == kModeApply;
         const bool same = !bmn && item.tl.ti == item.tl.tj;   // B half = A half
         const uint32_t idesc = bmn ? idesc_mn : idesc_k;
@@ -430,10 +511,34 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
       volatile int never = 0;
       mbar_wait_bounded(drain_bar, 0, &never, 10ull * 1000ull * 1000ull);
     }
-  } else if (warp < 2 + kEpiWarps) {
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ signal
+    // Publishes each item once all epilogue warps of this CTA have stored
+    // it: gpu-scope fence, then a release add on the item's phase counter.
+    if (lane == 0) {
+      int lt = 0;
+      uint4 nx = load_item_raw(p, pair);
+      for (int g = pair; g < total; g += npairs, ++lt) {
+        const MegaItem item = unpack_item(nx);
+        nx = load_item_raw(p, g + npairs);
+        if (!item_ok(item, g)) break;
+        if (!mbar_wait_bounded(epi_bar(lt % Cfg::kEpiBars), (lt / Cfg::kEpiBars) & 1,
+                               abort_flag)) {
+          fail(kErrTimeoutEpilogue);
+          break;
+        }
+        // release at gpu scope, cumulative over the stores the barrier
+        // made visible to this thread
+        red_release_gpu_add(done_counter(p, item.tl.mat, item.k, item.mode), 1);
+        *sig_count = lt + 1;
+      }
+    }
+  }
+  } else {
+    regs_increase<kNsRegsEpilogue>();
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;
-    const int quad = warp & 3;
+    const int ew = warp - kEpiWarp0;
+    const int quad = warp & 3;   // the TMEM lane quadrant this warp may read
     const int half = ew >> 2;
     const int r_pair = static_cast<int>(rank) * 128 + quad * 32 + lane;
     // This warp's 32 x 32 bf16 staging block and its transpose (4 KB, also
@@ -449,8 +554,8 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
     // 64-byte row segments; the 16-byte chunks of a staged row are
     // XOR-swizzled by (row / 2) % 4, which keeps both the row writes and the
     // segment reads free of bank conflicts.
-    auto put_block = [&](__nv_bfloat16* dst, int ld, int max_r, int max_c, int row0_,
-                         int col0_, bool mirror, const float (&v)[32]) {
+    auto put_block = [&](__nv_bfloat16* dst, int ld, int rows_alloc, int max_r, int max_c,
+                         int row0_, int col0_, bool mirror, const float (&v)[32]) {
       uint4* srow = reinterpret_cast<uint4*>(stg_d) + lane * 4;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -466,12 +571,24 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
       }
       __syncwarp();
       const int c = lane & 3;
+      // Device-checked build: every 8-element piece stays inside its row of
+      // the buffer (rows_alloc rows of ld elements), else it is skipped and
+      // the row recorded.
+      auto store_ok = [&](int gr, int gc) -> bool {
+        if constexpr (!kDeviceChecks) {
+          return true;
+        } else {
+          if (gr >= 0 && gr < rows_alloc && gc >= 0 && gc + 8 <= ld) return true;
+          record_check_failure(p.err, kErrCheckStore, gr);
+          return false;
+        }
+      };
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int rr = 8 * i + (lane >> 2);
         const uint4 val = reinterpret_cast<const uint4*>(stg_d)[rr * 4 + (c ^ ((rr >> 1) & 3))];
         const int gr = row0_ + rr, gc = col0_ + 8 * c;
-        if (gr < max_r && gc < max_c)
+        if (gr < max_r && gc < max_c && store_ok(gr, gc))
           *reinterpret_cast<uint4*>(dst + static_cast<size_t>(gr) * ld + gc) = val;
       }
       if (mirror) {
@@ -480,7 +597,7 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
           const int rr = 8 * i + (lane >> 2);
           const uint4 val = reinterpret_cast<const uint4*>(stg_m)[rr * 4 + c];
           const int gr = col0_ + rr, gc = row0_ + 8 * c;
-          if (gr < max_c && gc < max_r)
+          if (gr < max_c && gc < max_r && store_ok(gr, gc))
             *reinterpret_cast<uint4*>(dst + static_cast<size_t>(gr) * ld + gc) = val;
         }
       }
@@ -500,8 +617,11 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
     };
     constexpr int kLastCc = kPairTile / 32 - 2;   // cc of a warp's last block
     int lt = 0;
+    uint4 nx = load_item_raw(p, pair);
     for (int g = pair; g < total; g += npairs, ++lt) {
-      const MegaItem item = mega_item(p, g);
+      const MegaItem item = unpack_item(nx);
+      nx = load_item_raw(p, g + npairs);
+      if (!item_ok(item, g)) break;
       const NsTile tl = item.tl;
       const MatDev* md = p.mats + tl.mat;
       const int acc = lt & 1;
@@ -517,14 +637,17 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
       // waiting for it: the last step's W blocks, the poly's rows of A.
       float wa[32], wb[32];
       uint4 ar0[4], ar1[4];
+      // The first step's products carry the Frobenius scale (gram s^2, apply
+      // s), summed from the partials while the tensor cores run.
+      const float s = first && item.mode != kModePoly
+                          ? frob_scale(p.partials, md, lane, p.eps_frob) : 1.f;
       if (item.mode == kModeApply && last) {
         load_w_block(md, row0, colw, lane, wa);
         load_w_block(md, row0, colw + 64, lane, wb);
       } else if (item.mode == kModePoly) {
         // The generic reads of A need the gram stores of other CTAs.
         if (lane == 0) {
-          int32_t target = 2 * md->n_sym_tiles;
-          if (!wait_count(done_counter(p, tl.mat, item.k, kModeGram), target,
+          if (!wait_count(done_counter(p, tl.mat, item.k, kModeGram), item.dep_target,
                           abort_flag, p.err))
             fail(kErrTimeoutEpilogue);
         }
@@ -539,7 +662,6 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * kPairTile);
-      const float s = first ? p.mat_scale[tl.mat] : 1.f;
 
       if (item.mode == kModeGram || item.mode == kModePoly) {
         const bool diag_tile = tl.ti == tl.tj;
@@ -573,7 +695,7 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] *= mul;
           }
-          put_block(poly ? md->b : md->a, md->lda, m, m, row0, col0, !diag_tile, v);
+          put_block(poly ? md->b : md->a, md->lda, m, m, m, row0, col0, !diag_tile, v);
         };
         block(0, ar0, ar1);
         block(1, ar1, ar0);
@@ -590,7 +712,7 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] *= s;
           }
-          put_block(md->x[(item.k & 1) ^ 1], md->ldx, m, md->n, row0, col0, false, v);
+          put_block(md->x[(item.k & 1) ^ 1], md->ldx, m, m, md->n, row0, col0, false, v);
         }
       } else {
         // W <- W (1 - lr wd) - lr scale O over this warp's four blocks; the
@@ -607,7 +729,7 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] *= s;
           }
-          store_w_block(md, row0, colw + 64 * j, lane, decay, step, wv, v, stage_f32);
+          store_w_block(md, row0, colw + 64 * j, lane, decay, step, wv, v, stage_f32, p.err);
           if (j < 2) load_w_block(md, row0, colw + 64 * (j + 2), lane, wv);
         };
         block(0, wa);
@@ -636,25 +758,6 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
         if (ok) mbar_arrive(epi_bar(lt % Cfg::kEpiBars));
       }
       if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
-    }
-  } else {
-    // ------------------------------------------------------------ signal
-    // Publishes each item once all epilogue warps of this CTA have stored
-    // it: gpu-scope fence, then a release add on the item's phase counter.
-    if (lane == 0) {
-      int lt = 0;
-      for (int g = pair; g < total; g += npairs, ++lt) {
-        const MegaItem item = mega_item(p, g);
-        if (!mbar_wait_bounded(epi_bar(lt % Cfg::kEpiBars), (lt / Cfg::kEpiBars) & 1,
-                               abort_flag)) {
-          fail(kErrTimeoutEpilogue);
-          break;
-        }
-        // release at gpu scope, cumulative over the stores the barrier
-        // made visible to this thread
-        red_release_gpu_add(done_counter(p, item.tl.mat, item.k, item.mode), 1);
-        *sig_count = lt + 1;
-      }
     }
   }
 

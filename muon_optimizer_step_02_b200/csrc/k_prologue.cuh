@@ -19,6 +19,7 @@
 #include <cuda_bf16.h>
 
 #include "muon_types.cuh"
+#include "sm100_ptx.cuh"
 
 namespace muonb200 {
 
@@ -179,10 +180,19 @@ __global__ void __launch_bounds__(kProThreads, kOnePass ? 2 : 3)
 muon_prologue_kernel(const MatDev* __restrict__ mats,
                      const ProItem* __restrict__ items, int n_items, HyperDev h,
                      float* __restrict__ partials, int32_t* __restrict__ zero, int n_zero,
-                     int prefetch) {
+                     int prefetch, int write_lr, int32_t* err, int n_mats, int n_parts) {
   extern __shared__ __align__(16) unsigned char pro_smem[];
   __shared__ float warp_sums[kProThreads / 32];
   __shared__ float row_sums[2][kProThreads / 32];
+
+  // The Newton-Schulz kernel launched next may get its CTAs resident as
+  // soon as this grid's blocks leave their SMs; it waits for this grid to
+  // complete before it reads anything written here.
+  grid_launch_dependents();
+  // A scheduled step's learning rate, for the Newton-Schulz kernel (which
+  // advances the step counter once every block here has read it).
+  if (write_lr && h.step && blockIdx.x == 0 && threadIdx.x == 0)
+    *h.lr_slot = linear_ramp(h.lr_v0, h.lr_v1, h.lr_t0, h.lr_t1, *h.step);
 
   // The step's Newton-Schulz completion counters start at zero: the previous
   // step's Newton-Schulz kernel finished before this launch, and this step's
@@ -193,6 +203,17 @@ muon_prologue_kernel(const MatDev* __restrict__ mats,
   for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
     __syncthreads();   // the previous item's staging and sums are consumed
     const ProItem it = items[idx];
+    if constexpr (kDeviceChecks) {
+      // Device-checked build: an item outside its matrix (or with a partial
+      // slot past the table) is skipped and recorded.
+      const bool valid = it.mat >= 0 && it.mat < n_mats && it.nrows > 0 && it.row0 >= 0 &&
+                         it.row0 + it.nrows <= mats[it.mat].rows && it.part >= 0 &&
+                         it.part < n_parts;
+      if (!valid) {
+        if (threadIdx.x == 0) record_check_failure(err, kErrCheckPrologue, idx);
+        continue;
+      }
+    }
     const MatDev& md = mats[it.mat];
     const int cols = md.cols;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -406,8 +427,10 @@ muon_prologue_kernel(const MatDev* __restrict__ mats,
 }
 
 // The Frobenius scale s = 1 / (||X~||_F + eps_frob) of every matrix from its
-// prologue partials: one warp per matrix, lane l adds slots l, l + 32, ...
-// and the warp's butterfly adds the lanes, the same order on every run.
+// prologue partials, for the step without Newton-Schulz iterations (the
+// Newton-Schulz kernel sums the partials itself, in the same order): one
+// warp per matrix, lane l adds slots l, l + 32, ... and the warp's butterfly
+// adds the lanes, the same order on every run.
 //
 // With a schedule, thread 0 of block 0 also resolves the step's learning
 // rate into *lr_slot and advances the step counter: every prologue block has

@@ -449,8 +449,12 @@ bool set_kernel_attributes(size_t pro_smem, size_t pro_smem_one) {
                           lim.pro_one, pro_smem_one);
 }
 
+// Launch configuration of the tensor-core kernel: clusters of two CTAs and,
+// with `pdl`, programmatic stream serialization (the kernel may start while
+// the prologue before it finishes; it waits for it in-kernel).  attr needs
+// two entries.
 cudaLaunchConfig_t pair_launch_config(int clusters, cudaStream_t st,
-                                      cudaLaunchAttribute* attr) {
+                                      cudaLaunchAttribute* attr, bool pdl) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters);
   cfg.blockDim = dim3(kNsThreads);
@@ -460,8 +464,10 @@ cudaLaunchConfig_t pair_launch_config(int clusters, cudaStream_t st,
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   return cfg;
 }
 
@@ -472,8 +478,8 @@ int query_max_clusters() {
     cudaGetLastError();
     return 0;
   }
-  cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = pair_launch_config(1, nullptr, attr);
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = pair_launch_config(1, nullptr, attr, false);
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, ns_mega_pair_kernel, &cfg) != cudaSuccess) {
     cudaGetLastError();
@@ -489,8 +495,10 @@ void fill_sched_matrix(SchedMatrix& s, const Geom& g) {
   s.tn = g.tn;
 }
 
-// prologue (which also zeroes the step's counters) -> Frobenius scale ->
-// Newton-Schulz (or the finisher for 0 steps).  Each launch is checked as it
+// prologue (which also zeroes the step's counters) -> Newton-Schulz, a
+// programmatic dependent of the prologue that sums the Frobenius partials
+// itself; or, with 0 steps, prologue -> Frobenius scale -> finisher.  Each
+// launch is checked as it
 // is made: if the runtime refuses one, nothing after it is enqueued (a later
 // kernel would otherwise run on partials and counters the refused one never
 // wrote) and MUON_ERR_CUDA is returned; the launches before it have run.
@@ -523,30 +531,35 @@ muon_status_t enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
   int32_t* done = sc.counters;
   auto launched = [] { return cudaGetLastError() == cudaSuccess; };
   nvtxRangePushA("muon.prologue");
+  // The first prologue launch resolves a scheduled learning rate for the
+  // Newton-Schulz kernel (with 0 steps the scale kernel does).
+  const int lr_by_prologue = ns_steps > 0 ? 1 : 0;
   if (t.n_one > 0)
     muon_prologue_kernel<true><<<static_cast<unsigned>(t.pro_grid[0]), kProThreads,
                                  t.pro_smem_one, st>>>(t.mats, t.items, t.n_one, hd,
                                                        sc.partials, sc.counters,
-                                                       sc.n_counters, t.pro_prefetch);
+                                                       sc.n_counters, t.pro_prefetch,
+                                                       lr_by_prologue, t.err, sc.n_mats,
+                                                       t.n_items);
   bool ok = launched();
   if (ok && t.n_items > t.n_one) {
     muon_prologue_kernel<false><<<static_cast<unsigned>(t.pro_grid[1]), kProThreads,
                                   t.pro_smem, st>>>(
         t.mats, t.items + t.n_one, t.n_items - t.n_one, hd, sc.partials, sc.counters,
-        sc.n_counters, 0);
+        sc.n_counters, 0, t.n_one > 0 ? 0 : lr_by_prologue, t.err, sc.n_mats, t.n_items);
     ok = launched();
   }
   nvtxRangePop();
   if (!ok) return MUON_ERR_CUDA;
   if (rec) rec->after(MUON_KIND_PROLOGUE);
-  nvtxRangePushA("muon.frobenius_scale");
-  muon_frob_scale_kernel<<<static_cast<unsigned>((sc.n_mats + 7) / 8), 256, 0, st>>>(
-      t.mats, sc.n_mats, sc.partials, hd, sc.mat_scale);
-  nvtxRangePop();
-  if (!launched()) return MUON_ERR_CUDA;
-  if (rec) rec->after(MUON_KIND_SCALE);
 
   if (ns_steps == 0) {
+    nvtxRangePushA("muon.frobenius_scale");
+    muon_frob_scale_kernel<<<static_cast<unsigned>((sc.n_mats + 7) / 8), 256, 0, st>>>(
+        t.mats, sc.n_mats, sc.partials, hd, sc.mat_scale);
+    nvtxRangePop();
+    if (!launched()) return MUON_ERR_CUDA;
+    if (rec) rec->after(MUON_KIND_SCALE);
     muon_final_noiter_kernel<<<static_cast<unsigned>(t.n_items), kProThreads, 0,
                                st>>>(t.mats, t.items, sc.mat_scale, h.lr, lr_dev,
                                      h.weight_decay);
@@ -557,10 +570,12 @@ muon_status_t enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
   MegaParams p{};
   p.mats = t.mats;
   p.items = t.sched;
-  p.mat_scale = sc.mat_scale;
+  p.partials = sc.partials;
+  p.step_inc = sched ? step_dev : nullptr;
   p.err = t.err;
   p.done = done;
   p.n_items = static_cast<int32_t>(t.n_sched);
+  p.n_mats = sc.n_mats;
   p.steps = ns_steps;
   p.fault = fault;
   p.fresh = fresh ? 1 : 0;
@@ -573,8 +588,8 @@ muon_status_t enqueue_step(const LaunchTables& t, const muon_hyper_t& h,
   p.lr_dev = lr_dev;
   p.wd = h.weight_decay;
   p.eps_frob = h.eps_frob;
-  cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = pair_launch_config(t.clusters, st, attr);
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = pair_launch_config(t.clusters, st, attr, true);
   // test hook 2: more dynamic shared memory than the kernel was set up for,
   // so that the runtime refuses the launch (no kernel runs)
   if (fault == 2) cfg.dynamicSmemBytes = kMegaSmemBytes + 64 * 1024;
@@ -606,21 +621,23 @@ const char* muon_status_string(muon_status_t s) {
     case MUON_ERR_CUDA: return "CUDA error";
     case MUON_ERR_TIMEOUT: return "device-side wait timed out";
     case MUON_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case MUON_ERR_DEVICE_CHECK: return "device-side bounds check failed";
   }
   return "unknown status";
 }
 
 int32_t muon_step_launches(int32_t ns_steps) {
-  // one prologue kernel (which also zeroes the step's counters), the
-  // Frobenius scale kernel, then one Newton-Schulz launch for all steps (or
-  // the 0-step finisher); no memset
-  return ns_steps < 0 ? 0 : 3;
+  // one prologue kernel (which also zeroes the step's counters), then one
+  // Newton-Schulz launch for all steps; with 0 steps the Frobenius scale
+  // kernel and the finisher; no memset
+  return ns_steps < 0 ? 0 : (ns_steps > 0 ? 2 : 3);
 }
 
 int32_t muon_plan_step_launches(const muon_plan_t* plan, int32_t ns_steps) {
   if (!plan || ns_steps < 0) return 0;
   const int n_items = static_cast<int>(plan->items.size());
-  return (plan->n_one > 0 ? 1 : 0) + (n_items > plan->n_one ? 1 : 0) + 2;
+  return (plan->n_one > 0 ? 1 : 0) + (n_items > plan->n_one ? 1 : 0) +
+         (ns_steps > 0 ? 1 : 2);
 }
 
 int32_t ema_update_launches(int32_t n_tensors) {
@@ -760,10 +777,16 @@ void muon_plan_destroy(muon_plan_t* plan) {
 }
 
 muon_status_t muon_plan_set_fault(muon_plan_t* plan, int32_t fault) {
-  if (!plan || fault < 0 || fault > 2) return MUON_ERR_INVALID_ARG;
+  if (!plan || fault < 0 || fault > 3) return MUON_ERR_INVALID_ARG;
+  // fault 3 hands the kernel an invalid work item: only a build that checks
+  // every item before touching memory may receive one
+  if (fault == 3 && !kDeviceChecks) return MUON_ERR_UNSUPPORTED;
   plan->fault = fault;
+  plan->sched_steps = -1;   // the next call uploads the list anew
   return MUON_OK;
 }
+
+int32_t muon_device_checks(void) { return kDeviceChecks ? 1 : 0; }
 
 muon_status_t muon_plan_set_timing(muon_plan_t* plan, int32_t enable) {
   if (!plan) return MUON_ERR_INVALID_ARG;
@@ -804,9 +827,9 @@ muon_status_t muon_get_last_error(muon_plan_t* plan, muon_stream_t stream) {
   if (cudaMemcpy(&word, plan->d_err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
     return MUON_ERR_CUDA;
   if (word != 0) {
-    cudaMemset(plan->d_err, 0, sizeof(int32_t));
+    cudaMemset(plan->d_err, 0, 2 * sizeof(int32_t));
     cudaDeviceSynchronize();
-    return MUON_ERR_TIMEOUT;
+    return (word & 0xF00) == 0x200 ? MUON_ERR_DEVICE_CHECK : MUON_ERR_TIMEOUT;
   }
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
@@ -887,12 +910,19 @@ muon_status_t step_impl(muon_plan_t* plan, const muon_matrix_t* mats,
                                        plan->sched_cap, plan->sgroups.data(),
                                        plan->sorder.data(), plan->scl.data());
     if (n < 0) return MUON_ERR_UNSUPPORTED;
-    if (cudaMemcpyAsync(plan->d_sched, plan->sched.data(), sizeof(SchedItem) * n,
-                        cudaMemcpyHostToDevice, st) != cudaSuccess) {
+    // test hook 3 (device-checked build only): the last item of the list gets
+    // a tile row past its matrix; the kernel must catch it before any access
+    SchedItem saved = plan->sched[n - 1];
+    if (plan->fault == 3) plan->sched[n - 1].ti = static_cast<uint16_t>(0xFFFF);
+    const cudaError_t ce = cudaMemcpyAsync(plan->d_sched, plan->sched.data(),
+                                           sizeof(SchedItem) * n, cudaMemcpyHostToDevice, st);
+    plan->sched[n - 1] = saved;
+    if (plan->fault == 3) plan->sched_steps = -1;   // (re-uploaded clean later)
+    if (ce != cudaSuccess) {
       plan->sched_steps = -1;
       return MUON_ERR_CUDA;
     }
-    plan->sched_steps = ns_steps;
+    if (plan->fault != 3) plan->sched_steps = ns_steps;
     plan->sched_len = n;
   }
 
@@ -992,9 +1022,24 @@ muon_status_t ema_update_batched(float* const* ema, const float* const* params,
     if (units == 0) continue;
     const long long want = (units + kEmaThreads - 1) / kEmaThreads;
     const unsigned grid = static_cast<unsigned>(std::min<long long>(want, 8ll * sms));
+    // programmatic stream serialization: the blocks may become resident
+    // before the previous kernel of the stream ends and wait for it in-kernel
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kEmaThreads);
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     nvtxRangePushA("muon.ema");
-    ema_update_kernel<<<grid, kEmaThreads, 0, st>>>(p);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, ema_update_kernel, p);
     nvtxRangePop();
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return MUON_ERR_CUDA;
+    }
   }
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;

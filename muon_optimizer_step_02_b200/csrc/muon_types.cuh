@@ -71,8 +71,9 @@ struct NsTile {
 };
 
 // One item of the persistent Newton-Schulz schedule: a pair tile of one
-// phase (gram, poly, apply) of one step of one matrix.
-struct SchedItem {
+// phase (gram, poly, apply) of one step of one matrix.  16 bytes, read with
+// one vector load.
+struct alignas(16) SchedItem {
   uint16_t mat;
   uint16_t ti;    // pair-tile row (256 rows)
   uint16_t tj;    // pair-tile column (256 columns)
@@ -80,7 +81,10 @@ struct SchedItem {
   uint8_t mode;   // kModeGram / kModePoly / kModeApply
   uint8_t k;      // Newton-Schulz step
   uint16_t pad;
+  int32_t dep_target;  // completion count of the phase the item reads (two
+                       // per tile, one from each CTA); 0: no dependency
 };
+static_assert(sizeof(SchedItem) == 16, "SchedItem is one 16-byte load");
 
 struct HyperDev {
   float mu, lr, wd, eps_row, eps_frob;
@@ -112,5 +116,26 @@ enum NsMode : int32_t { kModeGram = 0, kModePoly = 1, kModeApply = 2 };
 constexpr int32_t kErrTimeoutProducer = 0x101;
 constexpr int32_t kErrTimeoutMma = 0x102;
 constexpr int32_t kErrTimeoutEpilogue = 0x103;
+// Device-checked build (MUON_DEVICE_CHECKS): a Newton-Schulz work item
+// outside its matrix's tile grid, a store outside its buffer, a prologue work
+// item outside its matrix.  The word after the error word receives the
+// offending list position, row or item index.
+constexpr int32_t kErrCheckItem = 0x201;
+constexpr int32_t kErrCheckStore = 0x202;
+constexpr int32_t kErrCheckPrologue = 0x203;
+
+#ifdef MUON_DEVICE_CHECKS
+constexpr bool kDeviceChecks = true;
+#else
+constexpr bool kDeviceChecks = false;
+#endif
+
+#ifdef __CUDACC__
+// Records the first failed device check (code, then its index).
+__device__ __forceinline__ void record_check_failure(int32_t* err, int32_t code,
+                                                     int32_t index) {
+  if (atomicCAS(err, 0, code) == 0) atomicExch(err + 1, index);
+}
+#endif
 
 }  // namespace muonb200

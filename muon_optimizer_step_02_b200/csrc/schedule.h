@@ -41,6 +41,23 @@ inline int sched_group_index(int mat, int k, int mode, int steps) {
 
 inline int sched_ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Whether a work item lies inside its matrix's tile grid and carries the
+// K-block count and dependency target of its phase: m x n working shape
+// (m <= n), `steps` Newton-Schulz steps.  The device-checked build of the
+// tensor-core kernel calls it on every item it decodes, before any access.
+__host__ __device__ inline bool sched_item_valid(int mode, int k, int ti, int tj, int kt,
+                                                 int dep_target, int m, int n, int steps) {
+  if (mode < 0 || mode > 2 || k < 0 || k >= steps || m < 1 || n < m) return false;
+  const int t2 = (m + kPairTile - 1) / kPairTile, tn = (n + kPairTile - 1) / kPairTile;
+  if (ti < 0 || ti >= t2) return false;
+  if (mode == kModeApply ? (tj < 0 || tj >= tn) : (tj < ti || tj >= t2)) return false;
+  if (kt != (mode == kModeGram ? (n + kTileK - 1) / kTileK : (m + kTileK - 1) / kTileK))
+    return false;
+  const int sym = t2 * (t2 + 1) / 2, app = t2 * tn;
+  const int want = mode == kModeGram ? (k == 0 ? 0 : 2 * app) : 2 * sym;
+  return dep_target == want;
+}
+
 // Item cost in tensor-core cycles of one CTA pair (256 x 256 x 64 per K
 // block) plus a fixed per-item cost; the last step's apply also moves W.
 inline double sched_cost(const SchedMatrix& mm, int mode, int k, int steps) {
@@ -171,6 +188,7 @@ inline long long build_schedule(const SchedMatrix* mats, int n_mats, int steps,
           it.mode = static_cast<uint8_t>(mode);
           it.k = static_cast<uint8_t>(k);
           it.pad = 0;
+          it.dep_target = g.dep < 0 ? 0 : 2 * groups[g.dep].size;
           // simulation: in-order execution on cluster pos % clusters
           const int c = static_cast<int>(pos % clusters);
           const double start = cl_time[c] > dep_t ? cl_time[c] : dep_t;

@@ -21,6 +21,35 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// ------------------------------------------ programmatic dependent launch
+// Blocks the calling thread, held by the hardware (no polling), until every
+// grid this grid depends on programmatically has completed and its memory
+// operations are visible; returns at once when there is no such grid.  A
+// kernel launched with programmatic stream serialization calls it before
+// reading anything its predecessor in the stream writes.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allows the grid launched next in the stream with programmatic stream
+// serialization to start once every CTA of this grid has called this (or
+// exited); it still waits in grid_dependency_wait for this grid to finish.
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ------------------------------------------------ warpgroup register split
+// Every thread of the calling warpgroup lowers (raises) its register count
+// to N; an increase waits until the block has that many registers free.
+template <int N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count)

@@ -66,7 +66,7 @@ def test_constants(L):
     assert binding.status_string(0) == "ok"
     assert "timed out" in binding.status_string(-5)
     assert binding.status_string(-99) == "unknown status"
-    assert L.muon_step_launches(5) == 3
+    assert L.muon_step_launches(5) == 2
     assert L.muon_step_launches(0) == 3
     assert L.muon_plan_step_launches(None, 5) == 0
     assert L.ema_update_launches(278) == 1
@@ -124,3 +124,17 @@ def test_closed_plan_refuses_bound_calls(L):
         plan._live_handle()
     assert e.value.status == binding.MUON_ERR_INVALID_ARG
     plan.close()                         # closing twice is harmless
+
+
+def test_device_checked_build_loads_and_exports_the_same_calls(L):
+    """The MUON_DEVICE_CHECKS build of the same sources (built by
+    _build.build beside the default one) exports every declared function and
+    reports itself; the default build reports 0."""
+    assert L.muon_device_checks() == 0
+    C = ctypes.CDLL(binding.CHECKED_LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(C, n)]
+    assert not missing, missing
+    C.muon_device_checks.restype = ctypes.c_int32
+    assert C.muon_device_checks() == 1
+    C.muon_status_string.restype = ctypes.c_char_p
+    assert b"bounds check" in C.muon_status_string(-7)

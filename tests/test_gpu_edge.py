@@ -56,9 +56,9 @@ def test_prologue_variants_in_one_plan():
     """One-pass and two-pass prologue items in the same step."""
     w = wl.custom(PROLOGUE_ROWS, H, Q5, grad_std=1.0, wid=111)
     g = GpuMuon(w)
-    # both prologue kernels, the scale kernel, the Newton-Schulz kernel
-    assert g.plan.step_launches(5) == 4
-    assert GpuMuon(wl.custom([(24, 1000)], H, Q5)).plan.step_launches(5) == 3
+    # both prologue kernels and the Newton-Schulz kernel
+    assert g.plan.step_launches(5) == 3
+    assert GpuMuon(wl.custom([(24, 1000)], H, Q5)).plan.step_launches(5) == 2
     for step in range(2):
         check_step(g, step, list(range(w.n_mats)))
 

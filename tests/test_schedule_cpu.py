@@ -37,7 +37,11 @@ def run(exe, shapes, steps, clusters, group_bytes=-1.0, lag=0):
     res = subprocess.run([exe], input=inp, capture_output=True, text=True,
                          check=True)
     lines = res.stdout.strip().split("\n")
-    items = [tuple(int(v) for v in ln.split()) for ln in lines[:-1]]
+    items = [tuple(int(v) for v in ln.split()) for ln in lines[:-2]]
+    _, accepted, missed = lines[-2].split()
+    # the device-side item check accepts every item and catches every
+    # corruption of one
+    assert int(accepted) == len(items) and int(missed) == 0
     makespan = float(lines[-1].split()[1])
     return items, makespan
 
@@ -51,6 +55,14 @@ def expected_tiles(r, c):
 
 
 def check(items, shapes, steps):
+    # the completion count each item waits for: two per tile of the phase it
+    # reads (0 for the first gram, which reads the prologue's output)
+    for mat, mode, k, _ti, _tj, _kt, target in items:
+        sym, app, _, _ = expected_tiles(*shapes[mat])
+        want_t = 0 if (mode == 0 and k == 0) else \
+            2 * (len(app) if mode == 0 else len(sym))
+        assert target == want_t, (mat, mode, k, target, want_t)
+    items = [it[:6] for it in items]
     # completeness
     want = Counter()
     for mat, (r, c) in enumerate(shapes):
