@@ -15,8 +15,6 @@
 
 #include <cstdint>
 
-#include "sm100_ptx.cuh"
-
 namespace muonb200 {
 
 constexpr int kEmaMaxSegs = 320;  // 10 KB of kernel parameters
@@ -39,11 +37,6 @@ struct EmaParams {
 
 __global__ void __launch_bounds__(kEmaThreads)
 ema_update_kernel(const __grid_constant__ EmaParams p) {
-  // Launched with programmatic stream serialization: the blocks may become
-  // resident while the previous kernel of the stream still runs (when it
-  // allows it) and wait here, held by the hardware, until it has completed
-  // -- the parameters may be the weights it writes.
-  grid_dependency_wait();
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   const long long u0 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   // last segment with ubeg <= u0

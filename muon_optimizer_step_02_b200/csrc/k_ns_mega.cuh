@@ -342,10 +342,10 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
   // set-up above overlaps the prologue's last blocks; everything below reads
   // what the prologue wrote (X~, the Frobenius partials, the zeroed
   // counters, the scheduled learning rate), so every thread waits for it to
-  // complete here.  The EMA launched after this kernel may then get its
-  // blocks resident; they wait in turn for this grid to finish.
+  // complete here.  (It lets no kernel after it start early: measured on the
+  // 11L step, EMA blocks waiting resident beside this kernel cost it 15-30
+  // us.)
   grid_dependency_wait();
-  grid_launch_dependents();
   // The prologue has read the scheduled step number; advance it once.
   if (p.step_inc != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.step_inc += 1;
   const uint32_t peer_abort = mapa_shared(smem_addr(const_cast<int*>(abort_flag)), rank ^ 1u);
@@ -636,7 +636,7 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
       // Inputs that do not depend on the accumulator are requested before
       // waiting for it: the last step's W blocks, the poly's rows of A.
       float wa[32], wb[32];
-      uint4 ar0[4], ar1[4];
+      uint4 ar[4][4];
       // The first step's products carry the Frobenius scale (gram s^2, apply
       // s), summed from the partials while the tensor cores run.
       const float s = first && item.mode != kModePoly
@@ -652,8 +652,12 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
             fail(kErrTimeoutEpilogue);
         }
         __syncwarp();
-        if (row_ok)
-          load_row32_bf16_raw(md->a + static_cast<size_t>(row) * md->lda, colw, m, ar0);
+        // this lane's row of A under all four blocks
+        if (row_ok) {
+          const __nv_bfloat16* arow = md->a + static_cast<size_t>(row) * md->lda;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) load_row32_bf16_raw(arow, colw + 64 * j, m, ar[j]);
+        }
       }
       if (!mbar_wait_bounded(tfull_bar(acc), aph, abort_flag)) {
         fail(kErrTimeoutEpilogue);
@@ -670,13 +674,10 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
         const float mul = poly ? p.c[item.k] : s * s;
         const float pb = p.b[item.k];
         const float pa = p.a[item.k];
-        // Block j (columns colw + 64 j) with A rows in `cur`; the next
-        // block's A rows are requested into `nxt` first.
-        auto block = [&](int j, const uint4 (&cur)[4], uint4 (&nxt)[4]) {
+        // Block j (columns colw + 64 j) with this lane's A row in `cur`.
+        auto block = [&](int j, const uint4 (&cur)[4]) {
           const int cc = half + 2 * j;
           const int col0 = colw + 64 * j;
-          if (poly && j < 3 && row_ok)
-            load_row32_bf16_raw(md->a + static_cast<size_t>(row) * md->lda, col0 + 64, m, nxt);
           float v[32];
           tmem_load_32cols(tbase + cc * 32, v);
           if (j == 3) release_acc(acc);
@@ -697,10 +698,10 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
           }
           put_block(poly ? md->b : md->a, md->lda, m, m, m, row0, col0, !diag_tile, v);
         };
-        block(0, ar0, ar1);
-        block(1, ar1, ar0);
-        block(2, ar0, ar1);
-        block(3, ar1, ar0);
+        block(0, ar[0]);
+        block(1, ar[1]);
+        block(2, ar[2]);
+        block(3, ar[3]);
       } else if (!last) {
 #pragma unroll 1
         for (int cc = half; cc < kPairTile / 32; cc += 2) {

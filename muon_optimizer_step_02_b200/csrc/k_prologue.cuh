@@ -186,8 +186,9 @@ muon_prologue_kernel(const MatDev* __restrict__ mats,
   __shared__ float row_sums[2][kProThreads / 32];
 
   // The Newton-Schulz kernel launched next may get its CTAs resident as
-  // soon as this grid's blocks leave their SMs; it waits for this grid to
-  // complete before it reads anything written here.
+  // soon as this grid's blocks leave their SMs (it needs a whole SM's shared
+  // memory); it waits for this grid to complete before it reads anything
+  // written here.
   grid_launch_dependents();
   // A scheduled step's learning rate, for the Newton-Schulz kernel (which
   // advances the step counter once every block here has read it).

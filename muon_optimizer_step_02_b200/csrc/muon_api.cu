@@ -1022,24 +1022,9 @@ muon_status_t ema_update_batched(float* const* ema, const float* const* params,
     if (units == 0) continue;
     const long long want = (units + kEmaThreads - 1) / kEmaThreads;
     const unsigned grid = static_cast<unsigned>(std::min<long long>(want, 8ll * sms));
-    // programmatic stream serialization: the blocks may become resident
-    // before the previous kernel of the stream ends and wait for it in-kernel
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kEmaThreads);
-    cfg.stream = st;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     nvtxRangePushA("muon.ema");
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, ema_update_kernel, p);
+    ema_update_kernel<<<grid, kEmaThreads, 0, st>>>(p);
     nvtxRangePop();
-    if (e != cudaSuccess) {
-      cudaGetLastError();
-      return MUON_ERR_CUDA;
-    }
   }
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
