@@ -398,21 +398,29 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
         const NsTile tl = item.tl;
         const MatDev* md = p.mats + tl.mat;
         const int src = item.k & 1;
+        // A and B' hold their upper 256-blocks only: a K block of the A
+        // operand (or of the polynomial's B operand) that falls below the
+        // diagonal is loaded from the stored block above it as an MN-major
+        // box (tm_an / tm_bn), and the MMA reads that K block transposed.
         const CUtensorMap* tm_a;
         const CUtensorMap* tm_b;
+        const CUtensorMap* tm_an = nullptr;   // MN-major map of the A operand
         if (item.mode == kModeGram) {
           tm_a = &md->tm_xk[src];
           tm_b = tm_a;
         } else if (item.mode == kModePoly) {
           tm_a = &md->tm_a;
           tm_b = tm_a;
+          tm_an = &md->tm_an;
         } else {
           tm_a = &md->tm_b;
           tm_b = &md->tm_xn[src];
+          tm_an = &md->tm_bn;
         }
         if (p.fresh) {
           tensormap_acquire(tm_a);
           if (tm_b != tm_a) tensormap_acquire(tm_b);
+          if (tm_an != nullptr) tensormap_acquire(tm_an);
         }
         const int32_t* dep = dep_counter(p, item);
         if (dep != nullptr) {
@@ -440,9 +448,26 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
           if (leader)
             mbar_arrive_expect_tx(full_bar(s), same ? 2u * Cfg::kABytes : Cfg::kTxBytes);
           const uint32_t lfull = leader_full0 + 8u * s;
-          tma_load_2d_pair(sA(s), tm_a, lfull, kb * kTileK, arow);
-          if (item.mode != kModeApply) {
+          const int kblk = kb * kTileK / kPairTile;   // 256-block column of this K block
+          // (an MN-major half is two 64-column boxes, the second 8 KB on)
+          if (tm_an != nullptr && kblk < tl.ti) {
+            tma_load_2d_pair(sA(s), tm_an, lfull, arow, kb * kTileK);
+            tma_load_2d_pair(sA(s) + 64 * kTileK * 2, tm_an, lfull, arow + 64, kb * kTileK);
+          } else {
+            tma_load_2d_pair(sA(s), tm_a, lfull, kb * kTileK, arow);
+          }
+          if (item.mode == kModeGram) {
             if (!same) tma_load_2d_pair(sB(s), tm_b, lfull, kb * kTileK, bcol);
+          } else if (item.mode == kModePoly) {
+            if (!same) {
+              if (kblk < tl.tj) {
+                tma_load_2d_pair(sB(s), tm_an, lfull, bcol, kb * kTileK);
+                tma_load_2d_pair(sB(s) + 64 * kTileK * 2, tm_an, lfull, bcol + 64,
+                                 kb * kTileK);
+              } else {
+                tma_load_2d_pair(sB(s), tm_b, lfull, kb * kTileK, bcol);
+              }
+            }
           } else {
             tma_load_2d_pair(sB(s), tm_b, lfull, bcol, kb * kTileK);
             tma_load_2d_pair(sB(s) + 64 * kTileK * 2, tm_b, lfull, bcol + 64,
@@ -464,8 +489,7 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc_k = idesc_bf16_f32_pair(kPairTile, false);
-      constexpr uint32_t idesc_mn = idesc_bf16_f32_pair(kPairTile, true);
+
       int it = 0, lt = 0;
       bool ok = true;
       uint4 nx = load_item_raw(p, pair);
@@ -473,9 +497,8 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
         const MegaItem item = unpack_item(nx);
         nx = load_item_raw(p, g + npairs);
         if (!item_ok(item, g)) break;
-        const bool bmn = item.mode == kModeApply;
-        const bool same = !bmn && item.tl.ti == item.tl.tj;   // B half = A half
-        const uint32_t idesc = bmn ? idesc_mn : idesc_k;
+        const bool apply = item.mode == kModeApply;
+        const bool same = !apply && item.tl.ti == item.tl.tj;   // B half = A half
         const int acc = lt & 1;
         const uint32_t aph = (lt >> 1) & 1;
         if (!mbar_wait_bounded(tempty_bar(acc), aph ^ 1u, abort_flag)) {
@@ -494,12 +517,21 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
             break;
           }
           tc_fence_after();
+          // Operand major-ness of this K block (see the producer): X in the
+          // apply, and blocks of A or B' below the diagonal, are MN-major.
+          const int kblk = kb * kTileK / kPairTile;
+          const bool amn = item.mode != kModeGram && kblk < item.tl.ti;
+          const bool bmn = apply || (item.mode == kModePoly && kblk < item.tl.tj);
+          const uint32_t idesc = idesc_bf16_f32_pair(kPairTile, bmn, amn);
 #pragma unroll
           for (int kk = 0; kk < kTileK / 16; ++kk) {
-            const uint64_t adesc = smem_desc_sw128(sA(s) + kk * 32, 16, 1024);
+            const uint64_t adesc =
+                amn ? smem_desc_sw128(sA(s) + kk * 2048, 64 * kTileK * 2, 1024)
+                    : smem_desc_sw128(sA(s) + kk * 32, 16, 1024);
+            const uint32_t bbase = same ? sA(s) : sB(s);
             const uint64_t bdesc =
-                bmn ? smem_desc_sw128(sB(s) + kk * 2048, 64 * kTileK * 2, 1024)
-                    : smem_desc_sw128((same ? sA(s) : sB(s)) + kk * 32, 16, 1024);
+                bmn ? smem_desc_sw128(bbase + kk * 2048, 64 * kTileK * 2, 1024)
+                    : smem_desc_sw128(bbase + kk * 32, 16, 1024);
             umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           umma_commit_pair_mc(empty_bar(s), 0x3);
@@ -696,7 +728,7 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] *= mul;
           }
-          put_block(poly ? md->b : md->a, md->lda, m, m, m, row0, col0, !diag_tile, v);
+          put_block(poly ? md->b : md->a, md->lda, m, m, m, row0, col0, false, v);
         };
         block(0, ar[0]);
         block(1, ar[1]);

@@ -381,7 +381,9 @@ bool fill_workspace_fields(MatDev& d, const Geom& g, char* ws) {
   d.a = reinterpret_cast<__nv_bfloat16*>(ws + g.a_off);
   d.b = reinterpret_cast<__nv_bfloat16*>(ws + g.b_off);
   if (!encode_bf16_2d(&d.tm_a, d.a, g.m, g.m, g.lda, kTileK, kTileM) ||
-      !encode_bf16_2d(&d.tm_b, d.b, g.m, g.m, g.lda, kTileK, kTileM))
+      !encode_bf16_2d(&d.tm_b, d.b, g.m, g.m, g.lda, kTileK, kTileM) ||
+      !encode_bf16_2d(&d.tm_an, d.a, g.m, g.m, g.lda, 64, kTileK) ||
+      !encode_bf16_2d(&d.tm_bn, d.b, g.m, g.m, g.lda, 64, kTileK))
     return false;
   d.rows = g.rows;
   d.cols = g.cols;

@@ -36,6 +36,8 @@ struct alignas(64) MatDev {
   CUtensorMap tm_xn[2];  // X ping/pong as an MN-major operand, box 64 x 64
   CUtensorMap tm_a;      // A = X X^T (m x m), box 64 x 128
   CUtensorMap tm_b;      // B = b A + c A A (m x m), box 64 x 128
+  CUtensorMap tm_an;     // A as an MN-major operand, box 64 x 64
+  CUtensorMap tm_bn;     // B as an MN-major operand, box 64 x 64
   __nv_bfloat16* x[2];   // m x ldx each
   __nv_bfloat16* a;      // m x lda
   __nv_bfloat16* b;      // m x lda

@@ -338,10 +338,12 @@ __device__ __forceinline__ void umma_commit_pair_mc(uint32_t bar, uint16_t mask)
       : "memory");
 }
 
-// Instruction descriptor, kind::f16 with bf16 A/B and fp32 D, M = 256 (pair).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32_pair(int n, bool b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
-         (static_cast<uint32_t>(n >> 3) << 17) |
+// Instruction descriptor, kind::f16 with bf16 A/B and fp32 D, M = 256 (pair);
+// bit 15 marks an MN-major A operand, bit 16 an MN-major B operand.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_pair(int n, bool b_mn_major,
+                                                           bool a_mn_major = false) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+         ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(n >> 3) << 17) |
          (static_cast<uint32_t>(256 >> 4) << 24);
 }
 
