@@ -44,7 +44,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
 # PTX wrappers and tables, and the host-built schedule that orders its work)
 KERNEL_SOURCES = {
     "ns_mega_pair_kernel": ("k_ns_mega.cuh", "k_ns_common.cuh", "sm100_ptx.cuh",
-                            "muon_types.cuh", "schedule.h"),
+                            "muon_types.cuh", "schedule.h", "muon_api.cu"),
 }
 
 
