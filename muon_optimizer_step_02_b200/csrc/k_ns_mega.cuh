@@ -16,9 +16,10 @@
 // and a tile's epilogue overlaps the next item's loads and MMAs.
 //
 // Per item:
-//   gram  A  = s^2 X X^T   (upper pair tiles; off-diagonal ones also stored
-//                          mirrored, so A is complete for its consumers)
-//   poly  B' = a I + b A + c A A   (A symmetric, so A A = A A^T)
+//   gram  A  = s^2 X X^T   (upper pair tiles only: a consumer reads a block
+//                          below the diagonal as the transpose of the stored
+//                          block above it)
+//   poly  B' = a I + b A + c A A   (A symmetric, so A A = A A^T; upper tiles)
 //   apply X <- s B' X      (last step: W <- W (1 - lr wd) - lr scale O)
 // X <- a X + B X is evaluated as (a I + B) X: one product, and the bf16 copy
 // of B' holds a + B on its diagonal instead of the cancelling pair.
@@ -71,8 +72,9 @@ struct MegaParams {
 };
 
 // Shared memory: the operand ring (per stage 16 KB of A rows + 16 KB of B
-// columns), then per epilogue warp a 32 x 32 bf16 output block and its
-// transpose (TMA-store sources), then the barriers.
+// columns), then per epilogue warp a 4 KB staging block (a 32 x 32 bf16
+// output block, or the 32 x 32 fp32 block of the weight update), then the
+// barriers.
 struct MegaCfg {
   static constexpr int kABytes = 128 * kTileK * 2;
   static constexpr int kBBytes = (kPairTile / 2) * kTileK * 2;
@@ -573,21 +575,19 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
     const int quad = warp & 3;   // the TMEM lane quadrant this warp may read
     const int half = ew >> 2;
     const int r_pair = static_cast<int>(rank) * 128 + quad * 32 + lane;
-    // This warp's 32 x 32 bf16 staging block and its transpose (4 KB, also
-    // the fp32 staging block of the weight update).
+    // This warp's 4 KB staging area: a 32 x 32 bf16 output block, or the
+    // fp32 block of the weight update.
     __nv_bfloat16* stg_d = out_stage + ew * 2 * Cfg::kOutBlockElems;
-    __nv_bfloat16* stg_m = stg_d + Cfg::kOutBlockElems;
     float* stage_f32 = reinterpret_cast<float*>(stg_d);
     // Stores v (lane = row) as bf16 at rows row0_ .., columns col0_ .. of
     // dst (leading dimension ld; rows below max_r, 8-column chunks starting
-    // below max_c, which ld covers) and, if `mirror`, its transpose at rows
-    // col0_ .., columns row0_ .. (square dst).  The block goes through shared
+    // below max_c, which ld covers).  The block goes through shared
     // memory so that every global store instruction writes eight whole
     // 64-byte row segments; the 16-byte chunks of a staged row are
     // XOR-swizzled by (row / 2) % 4, which keeps both the row writes and the
     // segment reads free of bank conflicts.
     auto put_block = [&](__nv_bfloat16* dst, int ld, int rows_alloc, int max_r, int max_c,
-                         int row0_, int col0_, bool mirror, const float (&v)[32]) {
+                         int row0_, int col0_, const float (&v)[32]) {
       uint4* srow = reinterpret_cast<uint4*>(stg_d) + lane * 4;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -596,10 +596,6 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
         for (int i = 0; i < 4; ++i)
           h[i] = __floats2bfloat162_rn(v[8 * q + 2 * i], v[8 * q + 2 * i + 1]);
         srow[q ^ ((lane >> 1) & 3)] = *reinterpret_cast<uint4*>(h);
-      }
-      if (mirror) {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) stg_m[e * 32 + lane] = __float2bfloat16_rn(v[e]);
       }
       __syncwarp();
       const int c = lane & 3;
@@ -622,16 +618,6 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
         const int gr = row0_ + rr, gc = col0_ + 8 * c;
         if (gr < max_r && gc < max_c && store_ok(gr, gc))
           *reinterpret_cast<uint4*>(dst + static_cast<size_t>(gr) * ld + gc) = val;
-      }
-      if (mirror) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int rr = 8 * i + (lane >> 2);
-          const uint4 val = reinterpret_cast<const uint4*>(stg_m)[rr * 4 + c];
-          const int gr = col0_ + rr, gc = row0_ + 8 * c;
-          if (gr < max_c && gc < max_r && store_ok(gr, gc))
-            *reinterpret_cast<uint4*>(dst + static_cast<size_t>(gr) * ld + gc) = val;
-        }
       }
       __syncwarp();   // staging free for the next block
     };
@@ -728,7 +714,7 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] *= mul;
           }
-          put_block(poly ? md->b : md->a, md->lda, m, m, m, row0, col0, false, v);
+          put_block(poly ? md->b : md->a, md->lda, m, m, m, row0, col0, v);
         };
         block(0, ar[0]);
         block(1, ar[1]);
@@ -745,7 +731,7 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] *= s;
           }
-          put_block(md->x[(item.k & 1) ^ 1], md->ldx, m, m, md->n, row0, col0, false, v);
+          put_block(md->x[(item.k & 1) ^ 1], md->ldx, m, m, md->n, row0, col0, v);
         }
       } else {
         // W <- W (1 - lr wd) - lr scale O over this warp's four blocks; the
