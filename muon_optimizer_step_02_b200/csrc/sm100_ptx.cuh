@@ -104,19 +104,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar,
 }
 
 // ---------------------------------------------------------------- TMA
-// 2-D tiled bulk tensor load global -> shared, completion counted on `bar`.
-// x is the innermost coordinate (elements); callers keep x * elem_size a
-// multiple of 16 bytes.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm,
-                                            uint32_t bar, int32_t x,
-                                            int32_t y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::"
-      "bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(x), "r"(y)
-      : "memory");
-}
-
 // Orders a tensor map written through the generic proxy (here: a host copy
 // into the plan's table) before its use by the tensor-map proxy.
 __device__ __forceinline__ void tensormap_acquire(const CUtensorMap* tm) {
@@ -125,60 +112,13 @@ __device__ __forceinline__ void tensormap_acquire(const CUtensorMap* tm) {
                : "memory");
 }
 
-__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* tm) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm))
-               : "memory");
-}
-
 // ---------------------------------------------------------------- tcgen05
-__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
-  asm volatile(
-      "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-          dst_smem),
-      "r"(ncols)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::
-                   : "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(
-                   taddr),
-               "r"(ncols)
-               : "memory");
-}
-
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
 
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// D[tmem] (+)= A[smem desc] * B[smem desc], bf16 inputs, fp32 accumulator.
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc,
-                                          uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(
-          d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrives once on `bar` when every tcgen05.mma issued so far by this thread
-// has completed.
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 "
-      "[%0];" ::"r"(bar)
-      : "memory");
 }
 
 // 32 lanes x 32 consecutive fp32 columns from TMEM, waited in the same asm
@@ -220,17 +160,6 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr,
   d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100
   d |= static_cast<uint64_t>(2) << 61;  // SWIZZLE_128B
   return d;
-}
-
-// Instruction descriptor, kind::f16 with bf16 A/B and fp32 D, M = 128.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int n, bool b_mn_major) {
-  return (1u << 4)                                  // D format: f32
-         | (1u << 7)                                // A format: bf16
-         | (1u << 10)                               // B format: bf16
-         | (0u << 15)                               // A K-major
-         | ((b_mn_major ? 1u : 0u) << 16)           // B major-ness
-         | (static_cast<uint32_t>(n >> 3) << 17)    // N / 8
-         | (static_cast<uint32_t>(128 >> 4) << 24); // M / 16
 }
 
 }  // namespace muonb200
@@ -338,8 +267,10 @@ __device__ __forceinline__ void umma_commit_pair_mc(uint32_t bar, uint16_t mask)
       : "memory");
 }
 
-// Instruction descriptor, kind::f16 with bf16 A/B and fp32 D, M = 256 (pair);
-// bit 15 marks an MN-major A operand, bit 16 an MN-major B operand.
+// Instruction descriptor, kind::f16 with bf16 A/B and fp32 D, M = 256 (pair):
+// D format f32 (bit 4), A and B bf16 (bits 7, 10), bit 15 an MN-major A
+// operand, bit 16 an MN-major B operand, N / 8 from bit 17, M / 16 from
+// bit 24.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32_pair(int n, bool b_mn_major,
                                                            bool a_mn_major = false) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
@@ -366,47 +297,6 @@ __device__ __forceinline__ void red_release_gpu_add(int32_t* p, int32_t v) {
 // accesses, in both directions.
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// Named barrier over `count` threads (ids 1..15; 0 is __syncthreads).
-__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
-}  // namespace muonb200
-
-// ---------------------------------------------------------------- TMA stores
-namespace muonb200 {
-
-// 2-D tiled bulk tensor store shared -> global (elements outside the tensor
-// are not written).  x is the innermost coordinate; x * elem_size % 16 == 0.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, uint32_t src,
-                                             int32_t x, int32_t y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(tm)),
-      "r"(src), "r"(x), "r"(y)
-      : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit_group() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// Wait until the committed bulk stores of this thread have read their
-// shared-memory source (the buffer may be rewritten).
-__device__ __forceinline__ void bulk_wait_group_read0() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-
-// Wait until the committed bulk stores of this thread are complete.
-__device__ __forceinline__ void bulk_wait_group0() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
-// Makes this thread's shared-memory writes visible to the async proxy (TMA).
-__device__ __forceinline__ void fence_proxy_async_shared() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 }  // namespace muonb200
