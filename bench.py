@@ -886,7 +886,8 @@ def main():
             dist.destroy_process_group()
     if line is None:
         return
-    if not args.no_cpu_baseline:
+    # the oracle's host-core baseline belongs to the one-GPU line only
+    if not args.no_cpu_baseline and world == 1:
         budget = float(os.environ.get("MUONB200_ORACLE_BUDGET_S", "15"))
         s, desc, threads = oracle_sample(load_workload(args.workload), budget)
         line["cpu_baseline"] = {"value": round(1.0 / s, 6), "unit": UNIT,
