@@ -63,10 +63,20 @@ class GpuMuon:
                        update_scales=self.scales, update_out=self.O)
 
 
+# An input on which bf16 arithmetic itself (the oracle's emulation of the
+# GPU path's rounding points) lands farther than TOL_O from fp64: the GPU may
+# be as far as that emulation, with this margin.
+EMU_MARGIN = 1.25
+
+
 def check_step(g: GpuMuon, step: int, idx, coeffs=None, emu_tol=None,
-               report=None):
+               report=None, o_tol_from_emu=False):
     """Runs one library step and compares the listed matrices with the fp64
-    oracle applied to the same pre-step state.  Returns the worst errors."""
+    oracle applied to the same pre-step state.  Returns the worst errors.
+    emu_tol: also compare O with the bf16-emulating oracle at this tolerance.
+    o_tol_from_emu: the fp64 bound on O is max(tol_o, EMU_MARGIN x the
+    emulation's own distance from fp64) -- for inputs outside the configs,
+    where bf16 arithmetic alone can exceed TOL_O (needs emu_tol)."""
     import torch
     w = g.w
     coeffs = w.coeffs if coeffs is None else coeffs
@@ -102,14 +112,19 @@ def check_step(g: GpuMuon, step: int, idx, coeffs=None, emu_tol=None,
         worst["W_e2e"] = max(worst["W_e2e"], e_we)
         worst["W_e2e_bound"] = max(worst["W_e2e_bound"], bound)
         assert np.all(np.isfinite(O1)), f"matrix {i}: non-finite update"
-        assert e_o <= tol_o(w.shapes[i]), \
-            f"matrix {i} {w.shapes[i]}: O error {e_o:.3e}"
+        Oe = None
+        o_bound = tol_o(w.shapes[i])
+        if emu_tol is not None:
+            _, _, Oe = mo.muon_step(W0[i], M0[i], Gh[i], hyp, coeffs,
+                                    g.scales[i], emulate_bf16=True)
+            if o_tol_from_emu:
+                o_bound = max(o_bound, EMU_MARGIN * rel_fro(Oe, Or))
+        assert e_o <= o_bound, \
+            f"matrix {i} {w.shapes[i]}: O error {e_o:.3e} (bound {o_bound:.3e})"
         assert e_m <= TOL_STATE, f"matrix {i}: momentum error {e_m:.3e}"
         assert e_wg <= TOL_STATE, f"matrix {i}: weight error {e_wg:.3e}"
         assert e_we <= bound * 1.01, f"matrix {i}: e2e weight {e_we:.3e}"
         if emu_tol is not None:
-            _, _, Oe = mo.muon_step(W0[i], M0[i], Gh[i], hyp, coeffs,
-                                    g.scales[i], emulate_bf16=True)
             e_emu = rel_fro(O1, Oe)
             worst["O_emu"] = max(worst["O_emu"], e_emu)
             assert e_emu <= emu_tol, f"matrix {i}: vs bf16 emulation {e_emu:.3e}"

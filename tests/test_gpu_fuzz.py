@@ -1,6 +1,14 @@
 """Seeded random cases against the fp64 oracle: random shapes (1..700 rows
 and columns, both orientations, aligned and not), random switches and step
-counts, several matrices per plan, two consecutive steps."""
+counts, several matrices per plan, two consecutive steps.  Each update is
+compared with the bf16-emulating oracle (the GPU path's rounding points) at
+1e-2 and with the fp64 oracle at 2e-2, or, on an input where bf16 arithmetic
+alone lands farther from fp64 (a 503 x 32 weight, working shape 32 x 503, at
+2.2e-2 and 2.6e-2), at 1.25 times that distance.  40 cases by
+default; MUONB200_FUZZ_CASES sets another count (and MUONB200_FUZZ_SEED0 the
+first seed) for longer runs."""
+import os
+
 import numpy as np
 import pytest
 
@@ -30,11 +38,15 @@ def _case(seed):
     return shapes, h, Q5[:k]
 
 
-@pytest.mark.parametrize("seed", list(range(40)))
+N_CASES = int(os.environ.get("MUONB200_FUZZ_CASES", "40"))
+SEED0 = int(os.environ.get("MUONB200_FUZZ_SEED0", "0"))
+
+
+@pytest.mark.parametrize("seed", list(range(SEED0, SEED0 + N_CASES)))
 def test_random_case_matches_oracle(seed):
     shapes, h, coeffs = _case(1000 + seed)
     w = wl.custom(shapes, h, coeffs, grad_std=float(10.0 ** (seed % 3 - 2)),
                   wid=600 + seed)
     g = GpuMuon(w)
     for step in range(2):
-        check_step(g, step, list(range(w.n_mats)))
+        check_step(g, step, list(range(w.n_mats)), emu_tol=1e-2, o_tol_from_emu=True)
