@@ -1,6 +1,7 @@
 """Seeded random cases against the fp64 oracle: random shapes (1..700 rows
 and columns, both orientations, aligned and not), random switches and step
-counts, several matrices per plan, two consecutive steps.  Each update is
+counts (the fixed quintic, or in about a third of the cases the committed
+4-step minimax table), several matrices per plan, two consecutive steps.  Each update is
 compared with the fp64 oracle at max(2e-2, 1.25 x the distance of the
 bf16-emulating oracle (the GPU path's rounding points) from fp64), and with
 that emulation at 1e-2 where the emulation is within 1.5e-2 of fp64.  Inputs
@@ -18,6 +19,7 @@ import pytest
 
 from gpu_harness import GpuMuon, check_step
 from muon_optimizer_step_02_b200 import workloads as wl
+from tables import polar_express_k4
 
 pytestmark = pytest.mark.gpu
 
@@ -42,6 +44,9 @@ def _case(seed):
                  lr=float(rng.uniform(0.005, 0.05)),
                  weight_decay=float(rng.uniform(0.0, 0.2)),
                  nesterov=bool(rng.random() < 0.8), eq_r=bool(rng.random() < 0.8))
+    # about a third of the cases take the committed 4-step minimax table
+    if rng.random() < 0.3:
+        return shapes, h, polar_express_k4()[:min(k, 4)]
     return shapes, h, Q5[:k]
 
 
