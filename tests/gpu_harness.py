@@ -64,7 +64,9 @@ class GpuMuon:
 
 
 # The distance of the oracle's bf16 emulation (the GPU path's rounding points)
-# from fp64 measures how sensitive an input is to rounding.  With
+# from fp64 measures how sensitive an input is to rounding (the pages give
+# no precision figure; the 2e-2 above holds on the five workloads, not on
+# every input a bf16 iteration can be handed).  With
 # o_tol_from_emu the GPU may be as far from fp64 as that emulation, with this
 # margin, and is held to the emulation itself only on inputs whose emulation
 # stays within EMU_SENSITIVE of fp64.
