@@ -15,12 +15,15 @@ NCCL (GPUs) and on gloo (CPU tests) alike:
   consecutive matrices, with the reduce-scatter of later buckets overlapping
   the step of earlier ones and each bucket's all-gather overlapping the
   steps after it (a communication stream beside the compute stream), and an
-  option to reduce the gradients in fp32.
+  option to reduce the gradients in fp32;
+* in both, an optional EMA of the weights each rank owns, updated by the
+  owner right after its step (the average shards like the momentum, with no
+  exchange of its own).
 
 Context: PR #1893 "Record: L_ParallelResiduals_UNetSkips_DepthRecur_Muon_
 1.0901", table "Architecture and training stack", row "Train context"
-(8-way distributed); PR #1396 section "Reproduction" (torchrun
---nproc_per_node=8).
+(8-way distributed) and row "EMA" (EMA_DECAY=0.9965); PR #1396 section
+"Reproduction" (torchrun --nproc_per_node=8).
 """
 
 from __future__ import annotations
@@ -123,20 +126,26 @@ class ShardLayout:
 
 
 def sharded_step_flat(layout: ShardLayout, W_flat, M_seg, G_flat, G_seg, rank,
-                      step_fn: Callable, group=None):
+                      step_fn: Callable, group=None, E_seg=None,
+                      ema_fn: Optional[Callable] = None):
     """One data-parallel Muon step on the flat layout:
       1. reduce-scatter the gradients: G_seg (seg elements) <- the sum over
          ranks of their G_flat segment for this rank;
       2. step this rank's matrices: step_fn(W_views, M_views, G_views) on
          views of its segment of W_flat, of M_seg and of G_seg;
+         with `ema_fn`, then ema_fn(E_views, W_views): the average of the
+         weights this rank owns, in E_seg (seg elements), from the updated
+         weights -- the EMA shards like the momentum, with no exchange;
       3. all-gather the updated segments of W_flat to every rank.
     Every rank issues the same two collectives."""
     import torch.distributed as dist
     dist.reduce_scatter_tensor(G_seg, G_flat, op=dist.ReduceOp.SUM, group=group)
     own = W_flat[rank * layout.seg:(rank + 1) * layout.seg]
     if layout.mine[rank]:
-        step_fn(layout.local_views(own, rank), layout.local_views(M_seg, rank),
-                layout.local_views(G_seg, rank))
+        w_views = layout.local_views(own, rank)
+        step_fn(w_views, layout.local_views(M_seg, rank), layout.local_views(G_seg, rank))
+        if ema_fn is not None:
+            ema_fn(layout.local_views(E_seg, rank), w_views)
     dist.all_gather_into_tensor(W_flat, own.clone(), group=group)
 
 
@@ -184,15 +193,17 @@ class BucketBuffers:
                            G_flat's dtype;
       G_step  seg          the gradients the step reads: G_seg itself when the
                            reduction is in the step's dtype, else a bf16 buffer
-                           that `to_step_dtype` fills from G_seg."""
+                           that `to_step_dtype` fills from G_seg;
+      E_seg   seg or None  the average (EMA) of the weights this rank owns."""
 
-    def __init__(self, W_flat, M_seg, G_flat, G_seg, G_step=None):
+    def __init__(self, W_flat, M_seg, G_flat, G_seg, G_step=None, E_seg=None):
         self.W_flat, self.M_seg, self.G_flat, self.G_seg = W_flat, M_seg, G_flat, G_seg
         self.G_step = G_seg if G_step is None else G_step
+        self.E_seg = E_seg
 
     @classmethod
     def allocate(cls, layout: ShardLayout, weight_dtype, grad_dtype, step_grad_dtype,
-                 device=None):
+                 device=None, with_ema=False):
         import torch
         W = torch.zeros(layout.numel(), dtype=weight_dtype, device=device)
         M = torch.zeros(layout.seg, dtype=weight_dtype, device=device)
@@ -200,12 +211,14 @@ class BucketBuffers:
         Gs = torch.zeros(layout.seg, dtype=grad_dtype, device=device)
         Gt = None if step_grad_dtype == grad_dtype else \
             torch.zeros(layout.seg, dtype=step_grad_dtype, device=device)
-        return cls(W, M, Gf, Gs, Gt)
+        E = torch.zeros(layout.seg, dtype=weight_dtype, device=device) if with_ema else None
+        return cls(W, M, Gf, Gs, Gt, E)
 
 
 def sharded_step_bucketed(layout: BucketedLayout, bufs: Sequence[BucketBuffers], rank: int,
                           step_fns: Sequence[Callable], group=None, comm_stream=None,
-                          to_step_dtype: Optional[Callable] = None):
+                          to_step_dtype: Optional[Callable] = None,
+                          ema_fns: Optional[Sequence[Callable]] = None):
     """One data-parallel Muon step over the buckets of `layout`.
 
       1. the reduce-scatters of every bucket's gradients are issued at once, in
@@ -215,8 +228,10 @@ def sharded_step_bucketed(layout: BucketedLayout, bufs: Sequence[BucketBuffers],
          reduce-scatter only, rounds the summed gradients to the step's dtype
          with `to_step_dtype(G_step, G_seg)` if the reduction ran in another
          dtype, and runs `step_fns[b](W_views, M_views, G_views)` on views of
-         this rank's segment; so bucket b's step overlaps the reduce-scatters
-         of the buckets after it;
+         this rank's segment, then, with `ema_fns`, ema_fns[b](E_views,
+         W_views) on its E_seg (the average of the weights it owns, no
+         exchange); so bucket b's step overlaps the reduce-scatters of the
+         buckets after it;
       3. the all-gathers of the updated weights are issued on `comm_stream` in
          bucket order, each waiting for its own bucket's step only, so that
          bucket b's all-gather overlaps the steps of the buckets after it;
@@ -247,8 +262,11 @@ def sharded_step_bucketed(layout: BucketedLayout, bufs: Sequence[BucketBuffers],
             to_step_dtype(bf.G_step, bf.G_seg)
         own = bf.W_flat[rank * L.seg:(rank + 1) * L.seg]
         if L.mine[rank]:
-            step_fns[b](L.local_views(own, rank), L.local_views(bf.M_seg, rank),
+            w_views = L.local_views(own, rank)
+            step_fns[b](w_views, L.local_views(bf.M_seg, rank),
                         L.local_views(bf.G_step, rank))
+            if ema_fns is not None:
+                ema_fns[b](L.local_views(bf.E_seg, rank), w_views)
         if comm_stream is not None:
             ev = torch.cuda.Event()
             ev.record(compute)

@@ -1,7 +1,8 @@
 """Multi-process host logic on CPU (gloo, world sizes 2 and 4): matrix
 ownership, the flat reduce-scatter / owner step / all-gather exchange of a
 sharded step, its bucketed form (with the gradient reduction in fp32 as an
-option), and the benchmark's max-over-ranks timing.  The per-rank compute is
+option, and each owner's EMA of its matrices), and the benchmark's
+max-over-ranks timing.  The per-rank compute is
 the fp64 oracle here; on GPUs it is the library's step."""
 import os
 import socket
@@ -54,6 +55,7 @@ def test_flat_layout_is_owner_ordered_and_aligned():
 
 
 SHARES = {2: [0.25, 0.75], 4: [0.125, 0.25, 0.25, 0.375]}
+EMA_D = 0.9965
 
 
 def _flat_worker(rank, world, port, q):
@@ -73,6 +75,9 @@ def _flat_worker(rank, world, port, q):
             v.copy_(torch.from_numpy(wl.weight(w, i).astype(np.float64)))
         M_seg = torch.zeros(L.seg, dtype=torch.float64)
         G_seg = torch.zeros(L.seg, dtype=torch.float64)
+        E_seg = torch.zeros(L.seg, dtype=torch.float64)
+        for j, v in zip(L.mine[rank], L.local_views(E_seg, rank)):
+            v.copy_(torch.from_numpy(wl.weight(w, j).astype(np.float64)))
         hyp = mo.MuonHyper(momentum=h.momentum, lr=h.lr, weight_decay=h.weight_decay)
 
         def step_fn(Wv, Mv, Gv):
@@ -81,6 +86,10 @@ def _flat_worker(rank, world, port, q):
                 a.copy_(torch.from_numpy(Wn))
                 m.copy_(torch.from_numpy(Mn))
 
+        def ema_fn(Ev, Wv):
+            for e, a in zip(Ev, Wv):
+                e.copy_(torch.from_numpy(mo.ema_update(e.numpy(), a.numpy(), EMA_D)))
+
         for step in range(2):
             G_flat = torch.zeros(L.numel(), dtype=torch.float64)
             # dyadic shares: the reduce-scatter sums them back to g exactly
@@ -88,9 +97,11 @@ def _flat_worker(rank, world, port, q):
             for i, v in enumerate(L.views(G_flat)):
                 g = wl.bf16_bits_to_f32(wl.grad_bits(w, i, step)).astype(np.float64)
                 v.copy_(torch.from_numpy(g * share))
-            sharding.sharded_step_flat(L, W_flat, M_seg, G_flat, G_seg, rank, step_fn)
+            sharding.sharded_step_flat(L, W_flat, M_seg, G_flat, G_seg, rank, step_fn,
+                                       E_seg=E_seg, ema_fn=ema_fn)
         t = sharding.max_over_ranks(1.0 + rank)
-        q.put((rank, [v.numpy().copy() for v in L.views(W_flat)], t))
+        E = {j: v.numpy().copy() for j, v in zip(L.mine[rank], L.local_views(E_seg, rank))}
+        q.put((rank, [v.numpy().copy() for v in L.views(W_flat)], t, E))
     finally:
         dist.destroy_process_group()
 
@@ -116,14 +127,23 @@ def test_flat_sharded_step_matches_single_process(world):
     hyp = mo.MuonHyper(momentum=h.momentum, lr=h.lr, weight_decay=h.weight_decay)
     W = [wl.weight(w, i).astype(np.float64) for i in range(len(shapes))]
     M = [np.zeros_like(x) for x in W]
+    E = [x.copy() for x in W]
     for step in range(2):
         for i in range(len(shapes)):
             G = wl.bf16_bits_to_f32(wl.grad_bits(w, i, step)).astype(np.float64)
             W[i], M[i], _ = mo.muon_step(W[i], M[i], G, hyp, coeffs, 1.0)
-    for rank, Ws, t in out:
+            E[i] = mo.ema_update(E[i], W[i], EMA_D)
+    owned = set()
+    for rank, Ws, t, Er in out:
         assert t == float(world)           # max over ranks of 1.0 + rank
         for a, b in zip(Ws, W):
             np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
+        # each rank's average covers exactly the matrices it owns
+        for j, e in Er.items():
+            np.testing.assert_allclose(e, E[j], rtol=1e-12, atol=1e-14)
+        assert not owned & set(Er)
+        owned |= set(Er)
+    assert owned == set(range(len(shapes)))
 
 
 SHAPES_B = [(48, 32), (32, 48), (40, 40), (16, 64), (64, 16), (24, 24), (8, 100),
@@ -140,10 +160,13 @@ def _bucket_worker(rank, world, port, q, n_buckets, fp32_reduce):
         w = wl.custom(SHAPES_B, h, coeffs, grad_std=1.0, wid=402)
         BL = sharding.BucketedLayout(SHAPES_B, world, n_buckets, 3)
         gdt = torch.float32 if fp32_reduce else torch.float64
-        bufs = [sharding.BucketBuffers.allocate(L, torch.float64, gdt, torch.float64)
+        bufs = [sharding.BucketBuffers.allocate(L, torch.float64, gdt, torch.float64,
+                                                with_ema=True)
                 for L in BL.layouts]
         for bk, L, bf in zip(BL.buckets, BL.layouts, bufs):
             for j, v in enumerate(L.views(bf.W_flat)):
+                v.copy_(torch.from_numpy(wl.weight(w, bk[j]).astype(np.float64)))
+            for j, v in zip(L.mine[rank], L.local_views(bf.E_seg, rank)):
                 v.copy_(torch.from_numpy(wl.weight(w, bk[j]).astype(np.float64)))
         hyp = mo.MuonHyper(momentum=h.momentum, lr=h.lr, weight_decay=h.weight_decay)
 
@@ -152,6 +175,10 @@ def _bucket_worker(rank, world, port, q, n_buckets, fp32_reduce):
                 Wn, Mn, _ = mo.muon_step(a.numpy(), m.numpy(), g.numpy(), hyp, coeffs, 1.0)
                 a.copy_(torch.from_numpy(Wn))
                 m.copy_(torch.from_numpy(Mn))
+
+        def ema_fn(Ev, Wv):
+            for e, a in zip(Ev, Wv):
+                e.copy_(torch.from_numpy(mo.ema_update(e.numpy(), a.numpy(), EMA_D)))
 
         def to_bf16_values(dst, src):
             # the library rounds the fp32 sum to bf16; the fp64 step reads it
@@ -166,12 +193,15 @@ def _bucket_worker(rank, world, port, q, n_buckets, fp32_reduce):
                     v.copy_(torch.from_numpy(g * share))
             sharding.sharded_step_bucketed(BL, bufs, rank, [step_fn] * n_buckets,
                                            to_step_dtype=to_bf16_values if fp32_reduce
-                                           else None)
+                                           else None, ema_fns=[ema_fn] * n_buckets)
         W = [None] * len(SHAPES_B)
+        E = {}
         for bk, L, bf in zip(BL.buckets, BL.layouts, bufs):
             for j, v in enumerate(L.views(bf.W_flat)):
                 W[bk[j]] = v.numpy().copy()
-        q.put((rank, W))
+            for j, v in zip(L.mine[rank], L.local_views(bf.E_seg, rank)):
+                E[bk[j]] = v.numpy().copy()
+        q.put((rank, W, E))
     finally:
         dist.destroy_process_group()
 
@@ -211,11 +241,19 @@ def test_bucketed_sharded_step_matches_single_process(world, n_buckets, fp32_red
     hyp = mo.MuonHyper(momentum=h.momentum, lr=h.lr, weight_decay=h.weight_decay)
     W = [wl.weight(w, i).astype(np.float64) for i in range(len(SHAPES_B))]
     M = [np.zeros_like(x) for x in W]
+    E = [x.copy() for x in W]
     for step in range(2):
         for i in range(len(SHAPES_B)):
             G = wl.bf16_bits_to_f32(wl.grad_bits(w, i, step)).astype(np.float64)
             W[i], M[i], _ = mo.muon_step(W[i], M[i], G, hyp, coeffs, 1.0)
-    for rank, Ws in out:
+            E[i] = mo.ema_update(E[i], W[i], EMA_D)
+    owned = set()
+    for rank, Ws, Er in out:
         for a, b in zip(Ws, W):
             # dyadic shares of bf16 values sum exactly in fp32 and in fp64
             np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
+        for j, e in Er.items():
+            np.testing.assert_allclose(e, E[j], rtol=1e-12, atol=1e-14)
+        assert not owned & set(Er)
+        owned |= set(Er)
+    assert owned == set(range(len(SHAPES_B)))
