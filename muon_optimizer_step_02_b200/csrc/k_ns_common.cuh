@@ -9,21 +9,25 @@
 
 namespace muonb200 {
 
-constexpr int kEpiWarps = 8;                 // two per TMEM lane quadrant
+constexpr int kEpiWarps = 12;                // three per TMEM lane quadrant
+constexpr int kEpiPerQuad = kEpiWarps / 4;
 // Warpgroup 0: producer warp, MMA warp, completion-signal warp, one idle
-// warp; warpgroups 1 and 2: the epilogue warps.
+// warp; warpgroups 1 to 3: the epilogue warps.
 constexpr int kEpiWarp0 = 4;                 // first epilogue warp
 constexpr int kNsThreads = 32 * (kEpiWarp0 + kEpiWarps);
 // Register split after set-up (setmaxnreg): the launch gives every thread
-// kNsRegsLaunch registers (384 threads x 168 = 64,512 of the SM's 65,536);
-// warpgroup 0 returns all but kNsRegsControl and the two epilogue
-// warpgroups take them, 128 x 56 + 256 x 224 = 64,512: the sum never
-// exceeds what the block was launched with, so the increase cannot wait.
-constexpr int kNsRegsLaunch = 168;
+// kNsRegsLaunch registers (512 threads x 128 = the SM's 65,536); warpgroup
+// 0 returns all but kNsRegsControl and the three epilogue warpgroups take
+// them, 128 x 56 + 384 x 152 = 65,536: the sum never exceeds what the block
+// was launched with, so the increase cannot wait.
+constexpr int kNsRegsLaunch = 128;
 constexpr int kNsRegsControl = 56;
-constexpr int kNsRegsEpilogue = 224;
-static_assert(128 * kNsRegsControl + 256 * kNsRegsEpilogue <= kNsThreads * kNsRegsLaunch,
+constexpr int kNsRegsEpilogue = 152;
+static_assert(128 * kNsRegsControl + 32 * kEpiWarps * kNsRegsEpilogue <=
+                  kNsThreads * kNsRegsLaunch,
               "register split exceeds the launch allocation");
+static_assert(kEpiWarps % 4 == 0 && 32 * kEpiWarps % 128 == 0,
+              "epilogue warps fill whole warpgroups, the same number per quadrant");
 
 
 

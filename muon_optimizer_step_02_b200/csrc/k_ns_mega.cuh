@@ -26,14 +26,16 @@
 // s = 1 / (||X~||_F + eps_frob) in step 0 (the Frobenius normalisation folded
 // into the first products), 1 afterwards.
 //
-// Roles (384 threads per CTA, three warpgroups): warp 0 issues TMA loads
-// (.cta_group::2, no multicast) into a 6-stage ring, counting both CTAs'
+// Roles (512 threads per CTA, four warpgroups): warp 0 issues TMA loads
+// (.cta_group::2, no multicast) into a 5-stage ring, counting both CTAs'
 // bytes on the leader's barrier; warp 1 of the leader issues the pair MMAs
 // from one thread and frees stages / hands over accumulators with multicast
-// tcgen05.commit; warp 2 publishes completed items; warp 3 idles; warps 4-11
-// (warpgroups 1 and 2) drain that CTA's 128 TMEM lanes and run the fused
-// epilogue.  After set-up warpgroup 0 gives its registers to the epilogue
-// warpgroups (setmaxnreg), which then hold their blocks without spilling.  All waits are bounded: a failure raises both CTAs' abort flags
+// tcgen05.commit; warp 2 publishes completed items; warp 3 idles; warps 4-15
+// (warpgroups 1 to 3, three warps per TMEM lane quadrant, each taking every
+// third 32-column block of the tile) drain that CTA's 128 TMEM lanes and run
+// the fused epilogue.  After set-up warpgroup 0 gives its registers to the
+// epilogue warpgroups (setmaxnreg), which then hold their blocks without
+// spilling.  All waits are bounded: a failure raises both CTAs' abort flags
 // and the global error word, and every CTA still meets the final cluster
 // barrier before TMEM is freed.
 //
@@ -53,7 +55,7 @@
 namespace muonb200 {
 
 constexpr int kMegaMaxSteps = 16;
-constexpr int kMegaStages = 6;
+constexpr int kMegaStages = 5;
 
 struct MegaParams {
   const MatDev* mats;
@@ -573,7 +575,9 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
     // ------------------------------------------------------------ epilogue
     const int ew = warp - kEpiWarp0;
     const int quad = warp & 3;   // the TMEM lane quadrant this warp may read
-    const int half = ew >> 2;
+    // this warp's 32-column blocks of the tile: cc = third, third + 3, ...
+    const int third = ew >> 2;
+    const int nb = (kPairTile / 32 - third + kEpiPerQuad - 1) / kEpiPerQuad;
     const int r_pair = static_cast<int>(rank) * 128 + quad * 32 + lane;
     // This warp's 4 KB staging area: a 32 x 32 bf16 output block, or the
     // fp32 block of the weight update.
@@ -633,7 +637,6 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
         else mbar_arrive_cluster_relaxed(leader_tempty0 + 8u * acc_);
       }
     };
-    constexpr int kLastCc = kPairTile / 32 - 2;   // cc of a warp's last block
     int lt = 0;
     uint4 nx = load_item_raw(p, pair);
     for (int g = pair; g < total; g += npairs, ++lt) {
@@ -650,18 +653,17 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
       const bool row_ok = row < m;
       const bool first = item.k == 0;
       const bool last = item.k == p.steps - 1;
-      const int colw = tl.tj * kPairTile + half * 32;   // this warp's first block
+      const int colw = tl.tj * kPairTile + third * 32;   // this warp's first block
       // Inputs that do not depend on the accumulator are requested before
       // waiting for it: the last step's W blocks, the poly's rows of A.
       float wa[32], wb[32];
-      uint4 ar[4][4];
+      uint4 ar[2][4];
       // The first step's products carry the Frobenius scale (gram s^2, apply
       // s), summed from the partials while the tensor cores run.
       const float s = first && item.mode != kModePoly
                           ? frob_scale(p.partials, md, lane, p.eps_frob) : 1.f;
       if (item.mode == kModeApply && last) {
         load_w_block(md, row0, colw, lane, wa);
-        load_w_block(md, row0, colw + 64, lane, wb);
       } else if (item.mode == kModePoly) {
         // The generic reads of A need the gram stores of other CTAs.
         if (lane == 0) {
@@ -670,11 +672,13 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
             fail(kErrTimeoutEpilogue);
         }
         __syncwarp();
-        // this lane's row of A under all four blocks
+        // this lane's row of A under the first two blocks (the third is
+        // requested once the first has been used)
         if (row_ok) {
           const __nv_bfloat16* arow = md->a + static_cast<size_t>(row) * md->lda;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) load_row32_bf16_raw(arow, colw + 64 * j, m, ar[j]);
+          for (int j = 0; j < 2; ++j)
+            load_row32_bf16_raw(arow, colw + 32 * kEpiPerQuad * j, m, ar[j]);
         }
       }
       if (!mbar_wait_bounded(tfull_bar(acc), aph, abort_flag)) {
@@ -692,13 +696,13 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
         const float mul = poly ? p.c[item.k] : s * s;
         const float pb = p.b[item.k];
         const float pa = p.a[item.k];
-        // Block j (columns colw + 64 j) with this lane's A row in `cur`.
+        // Block j (columns colw + 96 j) with this lane's A row in `cur`.
         auto block = [&](int j, const uint4 (&cur)[4]) {
-          const int cc = half + 2 * j;
-          const int col0 = colw + 64 * j;
+          const int cc = third + kEpiPerQuad * j;
+          const int col0 = colw + 32 * kEpiPerQuad * j;
           float v[32];
           tmem_load_32cols(tbase + cc * 32, v);
-          if (j == 3) release_acc(acc);
+          if (j == nb - 1) release_acc(acc);
           if (poly) {
             float av[32];
             unpack_row32_bf16(cur, av);
@@ -717,16 +721,18 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
           put_block(poly ? md->b : md->a, md->lda, m, m, m, row0, col0, v);
         };
         block(0, ar[0]);
+        if (poly && nb > 2 && row_ok)
+          load_row32_bf16_raw(md->a + static_cast<size_t>(row) * md->lda,
+                              colw + 2 * 32 * kEpiPerQuad, m, ar[0]);
         block(1, ar[1]);
-        block(2, ar[2]);
-        block(3, ar[3]);
+        if (nb > 2) block(2, ar[0]);
       } else if (!last) {
 #pragma unroll 1
-        for (int cc = half; cc < kPairTile / 32; cc += 2) {
+        for (int cc = third; cc < kPairTile / 32; cc += kEpiPerQuad) {
           const int col0 = tl.tj * kPairTile + cc * 32;
           float v[32];
           tmem_load_32cols(tbase + cc * 32, v);
-          if (cc >= kLastCc) release_acc(acc);
+          if (cc + kEpiPerQuad >= kPairTile / 32) release_acc(acc);
           if (first) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] *= s;
@@ -734,27 +740,28 @@ ns_mega_pair_kernel(const __grid_constant__ MegaParams p) {
           put_block(md->x[(item.k & 1) ^ 1], md->ldx, m, m, md->n, row0, col0, v);
         }
       } else {
-        // W <- W (1 - lr wd) - lr scale O over this warp's four blocks; the
-        // next block's W is already in registers (loaded two blocks ahead,
-        // the first two before the accumulator was ready).
+        // W <- W (1 - lr wd) - lr scale O over this warp's two or three
+        // blocks; each block's W is already in registers when it is stored
+        // (loaded one block ahead, the first before the accumulator was
+        // ready: two blocks ahead do not fit the 152-register budget).
         const float lr = p.lr_dev ? *p.lr_dev : p.lr;
         const float decay = 1.f - lr * p.wd;
         const float step = lr * md->update_scale;
         auto block = [&](int j, float (&wv)[32]) {
           float v[32];
-          tmem_load_32cols(tbase + (half + 2 * j) * 32, v);
-          if (j == 3) release_acc(acc);
+          tmem_load_32cols(tbase + (third + kEpiPerQuad * j) * 32, v);
+          if (j == nb - 1) release_acc(acc);
           if (first) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] *= s;
           }
-          store_w_block(md, row0, colw + 64 * j, lane, decay, step, wv, v, stage_f32, p.err);
-          if (j < 2) load_w_block(md, row0, colw + 64 * (j + 2), lane, wv);
+          store_w_block(md, row0, colw + 32 * kEpiPerQuad * j, lane, decay, step, wv, v,
+                        stage_f32, p.err);
+          if (j + 1 < nb) load_w_block(md, row0, colw + 32 * kEpiPerQuad * (j + 1), lane, wv);
         };
         block(0, wa);
-        block(1, wb);
-        block(2, wa);
-        block(3, wb);
+        block(1, wa);
+        if (nb > 2) block(2, wa);
       }
       // Hand the item to the signal warp (the arrival releases this warp's
       // stores to it).  Its barrier slot was last used four items ago; that
